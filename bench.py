@@ -1,0 +1,492 @@
+#!/usr/bin/env python3
+"""Benchmark of the KDA hot path on B200, one JSON line on rank 0.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                    [--workload prefill|varlen|extremes|decode|tiny_f32]
+
+A step is one pass of the whole hot path over one batch that is already
+resident in HBM: one ``kda_chunk_fwd`` over the workload (prefill workloads),
+or one ``kda_decode_step`` for all sequences (decode).  The default workload is
+the chunked prefill B=4, T=4096, H=16, dk=dv=128, bf16 q/k/v, fp32 gates and
+state, C=64.  Under torchrun every rank runs its own independent batch (a
+different seed) on its own GPU: the path shards by (sequence, head) with no
+exchange step, so there is no collective on the data path and scaling is weak.
+Timing: CUDA events on the stream the kernels run on, a barrier and a device
+synchronize on both sides of the timed region, the max over ranks.
+
+``--impl reference`` times the fp64 CPU oracle (the only reference this
+project has) on a bounded sample of the same workload, rank 0 only.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import re
+import statistics
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from gated_delta_rule_119_b200.inputs import (WORKLOADS, make_decode_state,  # noqa: E402
+                                             make_decode_step, make_inputs, make_workload,
+                                             to_torch)
+
+METRIC = ("KDA prefill tokens/s + TFLOP/s (% roofline) at dk=dv=128; "
+          "decode tokens/s, % HBM BW")
+PROFILES = os.path.join(ROOT, "profiles")
+KERNEL_SOURCES = {"chunk": "gated_delta_rule_119_b200/csrc/kda_chunk_tc.cu",
+                  "chunk_simt": "gated_delta_rule_119_b200/csrc/kda_chunk_simt.cuh",
+                  "decode": "gated_delta_rule_119_b200/csrc/kda_decode.cu"}
+
+
+# ------------------------------------------------------------ algorithmic work
+def alg_bytes_prefill(n_tok_heads: int, n_pairs: int, dk: int, dv: int, es: int,
+                      s0: bool, s_final: bool) -> int:
+    """Bytes the path must move: q, k, v, o in the input dtype, log_alpha and beta
+    fp32, plus one read (S0) and one write (S_final) of each dk x dv fp32 state."""
+    per_tok = es * (2 * dk + 2 * dv) + 4 * dk + 4
+    return n_tok_heads * per_tok + n_pairs * dk * dv * 4 * (int(s0) + int(s_final))
+
+
+def alg_flops_prefill(n_tok_heads: int, dk: int, dv: int, C: int = 64) -> int:
+    """Three state products (6 dk dv), the two causal C x C products counted on
+    their triangles (2 C (dk + dv)) and the C x C triangular solve (C^2 / 3)."""
+    return n_tok_heads * (6 * dk * dv + 2 * C * (dk + dv) + C * C // 3)
+
+
+def alg_bytes_decode(n_pairs: int, dk: int, dv: int, es: int) -> int:
+    return n_pairs * (2 * dk * dv * 4 + es * (2 * dk + 2 * dv) + 4 * dk + 4)
+
+
+# ----------------------------------------------------------- distributed plumbing
+def dist_env():
+    return (int(os.environ.get("RANK", 0)), int(os.environ.get("LOCAL_RANK", 0)),
+            int(os.environ.get("WORLD_SIZE", 1)))
+
+
+def rank_seed(base: int, rank: int) -> int:
+    """Each rank draws its own batch: weak scaling over independent problems."""
+    return base if rank == 0 else base * 1000 + rank
+
+
+def reduce_max(x: float, device) -> float:
+    import torch
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()):
+        return x
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def barrier(device=None):
+    import torch.distributed as dist
+    if dist.is_available() and dist.is_initialized():
+        if device is not None and getattr(device, "type", "cpu") == "cuda":
+            dist.barrier(device_ids=[device.index])
+        else:
+            dist.barrier()
+
+
+# ---------------------------------------------------------------- clock sampler
+class ClockSampler:
+    """Samples SM clock and clock-event reasons through NVML every `period` s."""
+
+    REASONS = {0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_cap",
+               0x8: "hw_slowdown", 0x10: "sync_boost", 0x20: "sw_thermal_slowdown",
+               0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown",
+               0x100: "display_clock_setting"}
+
+    def __init__(self, index: int, period: float = 0.01):
+        self.index, self.period = index, period
+        self.samples, self.reasons = [], set()
+        self.max_mhz = None
+        self._stop = threading.Event()
+        self._t = None
+        self.error = None
+
+    def __enter__(self):
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self._nv = pynvml
+            self._h = pynvml.nvmlDeviceGetHandleByIndex(self.index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self._h, pynvml.NVML_CLOCK_SM)
+        except Exception as e:  # pragma: no cover - no NVML
+            self.error = str(e)
+            return self
+        self._t = threading.Thread(target=self._run, daemon=True)
+        self._t.start()
+        return self
+
+    def _run(self):
+        nv = self._nv
+        while not self._stop.is_set():
+            try:
+                self.samples.append(nv.nvmlDeviceGetClockInfo(self._h, nv.NVML_CLOCK_SM))
+                mask = nv.nvmlDeviceGetCurrentClocksEventReasons(self._h)
+                for bit, name in self.REASONS.items():
+                    if mask & bit and name != "gpu_idle":
+                        self.reasons.add(name)
+            except Exception as e:  # pragma: no cover
+                self.error = str(e)
+                break
+            time.sleep(self.period)
+
+    def __exit__(self, *exc):
+        self._stop.set()
+        if self._t is not None:
+            self._t.join()
+        return False
+
+    def summary(self):
+        return {"sm_mhz": statistics.median(self.samples) if self.samples else None,
+                "sm_max_mhz": self.max_mhz, "reasons": sorted(self.reasons),
+                "samples": len(self.samples), "source": "NVML, every 10 ms during the timed region",
+                **({"error": self.error} if self.error else {})}
+
+
+# --------------------------------------------------------------- profile lookup
+def source_digest(rel: str) -> str:
+    with open(os.path.join(ROOT, rel), "rb") as f:
+        return hashlib.sha256(f.read()).hexdigest()[:16]
+
+
+def profiled_traffic(kernel_key: str, workload: str):
+    """DRAM bytes per launch recorded in a committed ncu summary, or None when
+    there is none or the kernel source changed since it was taken."""
+    path = os.path.join(PROFILES, f"traffic_{kernel_key}_{workload}.md")
+    if not os.path.exists(path):
+        return None
+    text = open(path).read()
+    m = re.search(r"dram_bytes_per_launch:\s*([0-9.eE+]+)", text)
+    h = re.search(r"kernel_source_sha256_16:\s*([0-9a-f]+)", text)
+    if not m or not h or h.group(1) != source_digest(KERNEL_SOURCES[kernel_key]):
+        return None
+    return float(m.group(1))
+
+
+def measured_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        p = json.load(open(path))
+        return p["hbm_gbs"], p["bf16_tflops"], "measured"
+    return 6650.0, 1590.0, "fallback"
+
+
+# ---------------------------------------------------------------- CPU baseline
+def cpu_baseline(inp, budget_s: float = 12.0):
+    """The fp64 oracle as it stands, on a bounded sample of (sequence, head)
+    pairs of the same workload, all host cores.  Tokens/s = token-heads / H / s."""
+    import oracle
+    cores = os.cpu_count() or 1
+    cu = inp.offsets()
+    lens = np.diff(cu)
+    order = [(n, h) for n in range(inp.n_seqs) for h in range(inp.H) if lens[n] > 0]
+    rng = np.random.default_rng(0)
+    rng.shuffle(order)
+    t = time.perf_counter()
+    oracle.recurrent(inp.q, inp.k, inp.v, inp.log_alpha, inp.beta, inp.S0, cu,
+                     tasks=order[:1], nthreads=1)
+    one = max(time.perf_counter() - t, 1e-6) / max(1, lens[order[0][0]])
+    # pairs that keep every core busy for about budget_s
+    per_pair = one * float(np.mean(lens))
+    n_pairs = int(max(1, min(len(order), round(budget_s * cores / per_pair))))
+    tasks = order[:n_pairs]
+    threads = min(cores, n_pairs)
+    t = time.perf_counter()
+    oracle.recurrent(inp.q, inp.k, inp.v, inp.log_alpha, inp.beta, inp.S0, cu, tasks=tasks,
+                     nthreads=threads)
+    dt = time.perf_counter() - t
+    tok_heads = int(sum(lens[n] for n, _ in tasks))
+    return {"value": tok_heads / inp.H / dt, "unit": "tokens/s", "cores": threads,
+            "kind": "oracle", "seconds": round(dt, 3),
+            "sample": f"{n_pairs} of {inp.n_seqs * inp.H} (sequence, head) pairs, "
+                      f"{tok_heads} token-heads, fp64 recurrence, {threads} threads"}
+
+
+def cpu_baseline_decode(ins, S0, budget_s: float = 12.0):
+    import oracle
+    cores = os.cpu_count() or 1
+    N, H = ins[0].q.shape[0], ins[0].q.shape[1]
+    steps = len(ins)
+    stack = lambda name: np.stack([getattr(i, name) for i in ins], axis=1).reshape(
+        N * steps, *getattr(ins[0], name).shape[1:])
+    cu = np.arange(N + 1) * steps
+    arrs = [stack(x) for x in ("q", "k", "v", "log_alpha", "beta")]
+    order = [(n, h) for n in range(N) for h in range(H)]
+    t = time.perf_counter()
+    oracle.recurrent(*arrs, S0, cu, tasks=order[:1], nthreads=1)
+    per_pair = max(time.perf_counter() - t, 1e-6)
+    n_pairs = int(max(1, min(len(order), round(budget_s * cores / per_pair))))
+    threads = min(cores, n_pairs)
+    t = time.perf_counter()
+    oracle.recurrent(*arrs, S0, cu, tasks=order[:n_pairs], nthreads=threads)
+    dt = time.perf_counter() - t
+    # a decode token is one sequence's step over all H heads
+    return {"value": n_pairs * steps / H / dt, "unit": "tokens/s", "cores": threads,
+            "kind": "oracle", "seconds": round(dt, 3),
+            "sample": f"{n_pairs} of {N * H} (sequence, head) states x {steps} steps, "
+                      f"fp64 recurrence, {threads} threads"}
+
+
+# -------------------------------------------------------------------- the runs
+def workload_config(name, inp_or_dims, n_gpus):
+    w = WORKLOADS[name]
+    cfg = {"workload": name, "B": w["B"], "T": w["T"], "H": w["H"], "dk": w["dk"],
+           "dv": w["dv"], "chunk": 64, "dtype": w["dtype"], "state_in": w["state"],
+           "varlen": w["varlen"], "gates": w["gates"],
+           "global_batch": w["B"] * n_gpus, "seq_len": w["T"],
+           "parallelism": f"dp{n_gpus}: independent batches per rank, no collective"}
+    return cfg
+
+
+def run_ours(args, rank, local_rank, world):
+    import torch
+    from gated_delta_rule_119_b200 import kda_chunk_fwd, kda_decode_step, load_library
+    load_library()
+    device = torch.device("cuda", local_rank)
+    torch.cuda.set_device(device)
+    name = args.workload
+    w = WORKLOADS[name]
+    hbm, bf16_tf, peak_kind = measured_peaks()
+    stream = torch.cuda.current_stream(device)
+    es = 2 if w["dtype"] == "bf16" else 4
+    launches_per_step = 1
+
+    if name == "decode":
+        N, H, dk, dv = w["B"], w["H"], w["dk"], w["dv"]
+        n_in = max(1, min(args.decode_inputs, args.steps + args.warmup))
+        ins = [make_decode_step(N, H, dk, dv, w["dtype"], rank_seed(w["index"], rank), t)
+               for t in range(n_in)]
+        S0 = make_decode_state(N, H, dk, dv, rank_seed(w["index"], rank))
+        dev_in = [to_torch(i, device) for i in ins]
+        S = torch.from_numpy(S0).to(device)
+        out = torch.empty((N, H, dv), dtype=dev_in[0]["q"].dtype, device=device)
+
+        def step(i):
+            d = dev_in[i % n_in]
+            kda_decode_step(d["q"], d["k"], d["v"], d["log_alpha"], d["beta"], S, out)
+        units_per_step = N                       # tokens (one per sequence)
+        bytes_per_launch = alg_bytes_decode(N * H, dk, dv, es)
+        flops_per_launch = N * H * 7 * dk * dv
+        kernel_key = "decode"
+        inp_for_cpu = None
+    else:
+        inp = make_workload(name) if rank == 0 else make_inputs(
+            w["B"], w["T"], w["H"], w["dk"], w["dv"], w["dtype"], rank_seed(w["index"], rank),
+            state=w["state"], varlen=w["varlen"], gates=w["gates"])
+        d = to_torch(inp, device)
+        out = torch.empty(d["v"].shape, dtype=d["q"].dtype, device=device)
+        Sf = torch.empty((inp.n_seqs, inp.H, inp.dk, inp.dv), dtype=torch.float32, device=device)
+
+        def step(i):
+            kda_chunk_fwd(d["q"], d["k"], d["v"], d["log_alpha"], d["beta"], d["S0"],
+                          d["cu_seqlens"], out, Sf)
+        tok_heads = inp.total_tokens * inp.H
+        units_per_step = inp.total_tokens
+        bytes_per_launch = alg_bytes_prefill(tok_heads, inp.n_seqs * inp.H, inp.dk, inp.dv, es,
+                                             inp.S0 is not None, True)
+        flops_per_launch = alg_flops_prefill(tok_heads, inp.dk, inp.dv)
+        kernel_key = "chunk_simt"
+        inp_for_cpu = inp
+
+    for i in range(args.warmup):
+        step(i)
+    torch.cuda.synchronize(device)
+    barrier(device)
+    torch.cuda.synchronize(device)
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with ClockSampler(device.index if device.index is not None else 0) as clk:
+        ev0.record(stream)
+        for i in range(args.steps):
+            step(args.warmup + i)
+        ev1.record(stream)
+        torch.cuda.synchronize(device)
+    barrier(device)
+    torch.cuda.synchronize(device)
+    ms_local = ev0.elapsed_time(ev1) / args.steps
+    ms = reduce_max(ms_local, device)
+
+    # per-launch duration of the dominant (only) kernel, events around each launch
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+           for _ in range(min(args.steps, 20))]
+    for i, (a, b) in enumerate(evs):
+        a.record(stream)
+        step(i)
+        b.record(stream)
+    torch.cuda.synchronize(device)
+    launch_ms = float(np.mean([a.elapsed_time(b) for a, b in evs]))
+    launch_ms = reduce_max(launch_ms, device)
+
+    # end to end through the public API with host buffers
+    e2e = run_e2e(args, name, device, stream, rank)
+
+    value = units_per_step * world / (ms / 1e3)
+    achieved = bytes_per_launch / (launch_ms / 1e3) / 1e9
+    traffic = profiled_traffic(kernel_key, name)
+    res = {
+        "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": w["dtype"], "data": "synthetic (seeded numpy; see inputs.py recipe)",
+        "config": {**workload_config(name, None, world),
+                   "l2": "no flush: the inputs of one step exceed the 126 MB L2"
+                   if bytes_per_launch > 126e6 else "inputs fit in L2; reported as is"},
+        "tflops": flops_per_launch / (launch_ms / 1e3) / 1e12,
+        "roofline": {"bound": "hbm", "achieved": achieved, "peak": hbm, "unit": "GB/s",
+                     "frac": achieved / hbm, "traffic": traffic,
+                     "peak_kind": f"{peak_kind} (STREAM-style copy, burst)",
+                     "kernel": kernel_key, "alg_bytes_per_launch": bytes_per_launch,
+                     "launch_ms": launch_ms},
+        "clocks": clk.summary(),
+        "e2e": e2e,
+        "gpu_launches": args.steps * launches_per_step,
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        if name == "decode":
+            res["cpu_baseline"] = cpu_baseline_decode(ins[:min(4, len(ins))], S0,
+                                                      args.cpu_budget)
+        else:
+            res["cpu_baseline"] = cpu_baseline(inp_for_cpu, args.cpu_budget)
+    return res
+
+
+def run_e2e(args, name, device, stream, rank):
+    """The same metric through the public call with pinned host buffers: H2D of
+    the step's inputs, the call, D2H of its results, all inside the timed region."""
+    import torch
+    from gated_delta_rule_119_b200 import kda_chunk_fwd, kda_decode_step
+    w = WORKLOADS[name]
+    steps = max(1, min(args.steps, args.e2e_steps))
+    if name == "decode":
+        N, H, dk, dv = w["B"], w["H"], w["dk"], w["dv"]
+        inp = make_decode_step(N, H, dk, dv, w["dtype"], rank_seed(w["index"], rank), 0)
+        host = to_torch(inp, "cpu", pin=True)
+        S_host = torch.from_numpy(make_decode_state(N, H, dk, dv, 5)).pin_memory()
+        out_host = torch.empty((N, H, dv), dtype=host["q"].dtype).pin_memory()
+        S_dev = torch.empty_like(S_host, device=device)
+        units = N
+    else:
+        inp = make_workload(name) if rank == 0 else make_inputs(
+            w["B"], w["T"], w["H"], w["dk"], w["dv"], w["dtype"], rank_seed(w["index"], rank),
+            state=w["state"], varlen=w["varlen"], gates=w["gates"])
+        host = to_torch(inp, "cpu", pin=True)
+        out_host = torch.empty(host["v"].shape, dtype=host["q"].dtype).pin_memory()
+        S_host = torch.empty((inp.n_seqs, inp.H, inp.dk, inp.dv), dtype=torch.float32).pin_memory()
+        units = inp.total_tokens
+    h2d = sum(t.numel() * t.element_size() for t in host.values() if t is not None)
+    if name == "decode":
+        h2d += S_host.numel() * 4
+    d2h = out_host.numel() * out_host.element_size() + S_host.numel() * 4
+
+    def one():
+        d = {k: (None if t is None else t.to(device, non_blocking=True)) for k, t in host.items()}
+        if name == "decode":
+            S_dev.copy_(S_host, non_blocking=True)
+            o = kda_decode_step(d["q"], d["k"], d["v"], d["log_alpha"], d["beta"], S_dev)
+            out_host.copy_(o, non_blocking=True)
+            S_host.copy_(S_dev, non_blocking=True)
+        else:
+            o, Sf = kda_chunk_fwd(d["q"], d["k"], d["v"], d["log_alpha"], d["beta"], d["S0"],
+                                  d["cu_seqlens"])
+            out_host.copy_(o, non_blocking=True)
+            S_host.copy_(Sf, non_blocking=True)
+
+    one()
+    torch.cuda.synchronize(device)
+    barrier(device)
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    ev0.record(stream)
+    for _ in range(steps):
+        one()
+    ev1.record(stream)
+    torch.cuda.synchronize(device)
+    ms = reduce_max(ev0.elapsed_time(ev1) / steps, device)
+    world = int(os.environ.get("WORLD_SIZE", 1))
+    return {"value": units * world / (ms / 1e3), "unit": "tokens/s", "ms_per_step": ms,
+            "steps": steps, "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
+            "path": "pinned host -> kda_* public call -> pinned host"}
+
+
+def run_reference(args, rank, world):
+    """The fp64 CPU oracle on a bounded sample of the same workload."""
+    name = args.workload
+    w = WORKLOADS[name]
+    samples = []
+    for i in range(args.warmup + args.steps):
+        if name == "decode":
+            N, H, dk, dv = w["B"], w["H"], w["dk"], w["dv"]
+            ins = [make_decode_step(N, H, dk, dv, w["dtype"], w["index"], t) for t in range(2)]
+            cb = cpu_baseline_decode(ins, make_decode_state(N, H, dk, dv, w["index"]),
+                                     args.ref_step_budget)
+        else:
+            if i == 0:
+                inp = make_workload(name)
+            cb = cpu_baseline(inp, args.ref_step_budget)
+        if i >= args.warmup:
+            samples.append(cb)
+    value = statistics.median(s["value"] for s in samples)
+    ms = float(np.median([s["seconds"] * 1e3 for s in samples]))
+    return {"impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s",
+            "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic (seeded numpy; see inputs.py recipe)",
+            "config": workload_config(name, None, 1),
+            "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": samples[-1]["cores"],
+                             "kind": "oracle", "sample": samples[-1]["sample"]},
+            "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0},
+            "gpu_launches": 0}
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", choices=sorted(WORKLOADS), default="prefill")
+    ap.add_argument("--e2e-steps", type=int, default=10)
+    ap.add_argument("--decode-inputs", type=int, default=64,
+                    help="distinct per-step decode inputs held on the device (cycled)")
+    ap.add_argument("--cpu-budget", type=float, default=12.0,
+                    help="seconds of host-core work for the CPU baseline sample")
+    ap.add_argument("--ref-step-budget", type=float, default=4.0)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args(argv)
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    rank, local_rank, world = dist_env()
+
+    if args.impl == "reference":
+        if rank == 0:
+            print(json.dumps(run_reference(args, rank, world)), flush=True)
+        return 0
+
+    import torch
+    import torch.distributed as dist
+    if world > 1:
+        from datetime import timedelta
+        torch.cuda.set_device(local_rank)
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120),
+                                device_id=torch.device("cuda", local_rank))
+    try:
+        res = run_ours(args, rank, local_rank, world)
+    finally:
+        if world > 1 and dist.is_initialized():
+            dist.destroy_process_group()
+    if rank == 0:
+        print(json.dumps(res), flush=True)
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,8 @@
+"""KDA (Kimi Delta Attention) on B200: chunked prefill and decode through the
+C ABI of libkda.so (include/kda.h).  Importing the package does not load the
+library; the first call does, and fails loudly if it is missing."""
+from .binding import (KDA_BF16, KDA_F32, KDAError, kda_chunk_fwd, kda_decode_step,
+                      kda_status_string, load_library)
+
+__all__ = ["KDA_BF16", "KDA_F32", "KDAError", "kda_chunk_fwd", "kda_decode_step",
+           "kda_status_string", "load_library"]

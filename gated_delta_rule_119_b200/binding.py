@@ -1,0 +1,161 @@
+"""Thin Python binding of libkda.so (ctypes).
+
+Argument marshalling only: every step of KDA runs in the library's CUDA
+kernels.  PyTorch supplies device memory and the current stream.  If the
+library is missing, :func:`load_library` raises; there is no fallback.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(HERE, "libkda.so")
+
+KDA_F32, KDA_BF16 = 0, 1
+STATUS = {0: "KDA_OK", -1: "KDA_ERR_NULL", -2: "KDA_ERR_DIM", -3: "KDA_ERR_CHUNK",
+          -4: "KDA_ERR_ALIGN", -5: "KDA_ERR_DTYPE", -6: "KDA_ERR_ALIAS", -7: "KDA_ERR_CUDA",
+          -8: "KDA_ERR_TIMEOUT"}
+EXPORTS = ("kda_chunk_fwd", "kda_decode_step", "kda_status_string")
+
+_lib = None
+
+
+class KDAError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        super().__init__(f"{where}: {kda_status_string(status)}")
+
+
+def load_library(path: str | None = None):
+    """Load libkda.so (built in-tree by ``gated_delta_rule_119_b200.build``)."""
+    global _lib
+    if _lib is not None and path is None:
+        return _lib
+    p = path or LIB_PATH
+    if not os.path.exists(p):
+        raise RuntimeError(f"libkda.so not found at {p}: build it with "
+                           "`python -m gated_delta_rule_119_b200.build` (nvcc, sm_100a)")
+    lib = ctypes.CDLL(p)
+    V, F, I32 = ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int
+    lib.kda_chunk_fwd.argtypes = [V, V, V, F, F, F, V, V, F] + [I32] * 7 + [V]
+    lib.kda_chunk_fwd.restype = ctypes.c_int
+    lib.kda_decode_step.argtypes = [V, V, V, F, F, F, V] + [I32] * 5 + [V]
+    lib.kda_decode_step.restype = ctypes.c_int
+    lib.kda_status_string.argtypes = [ctypes.c_int]
+    lib.kda_status_string.restype = ctypes.c_char_p
+    if path is None:
+        _lib = lib
+    return lib
+
+
+def kda_status_string(status: int) -> str:
+    return load_library().kda_status_string(int(status)).decode()
+
+
+# ----------------------------------------------------------------- raw ABI calls
+def chunk_fwd_raw(q, k, v, log_alpha, beta, S0, cu_seqlens, out, S_final, B, T, H, dk, dv,
+                  C, dtype, stream) -> int:
+    """Call the C entry point with integer addresses (0 = NULL)."""
+    return load_library().kda_chunk_fwd(q or None, k or None, v or None, log_alpha or None,
+                                        beta or None, S0 or None, cu_seqlens or None,
+                                        out or None, S_final or None, B, T, H, dk, dv, C,
+                                        dtype, stream or None)
+
+
+def decode_step_raw(q, k, v, log_alpha, beta, S_inout, out, N, H, dk, dv, dtype,
+                    stream) -> int:
+    return load_library().kda_decode_step(q or None, k or None, v or None, log_alpha or None,
+                                          beta or None, S_inout or None, out or None, N, H, dk,
+                                          dv, dtype, stream or None)
+
+
+# ------------------------------------------------------------ torch-facing calls
+def _torch():
+    import torch
+    return torch
+
+
+def _dtype_code(t) -> int:
+    torch = _torch()
+    if t.dtype == torch.float32:
+        return KDA_F32
+    if t.dtype == torch.bfloat16:
+        return KDA_BF16
+    raise TypeError(f"q/k/v must be float32 or bfloat16, got {t.dtype}")
+
+
+def _ptr(t):
+    return 0 if t is None else t.data_ptr()
+
+
+def _check(t, name, dtype=None):
+    if t is None:
+        return
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if dtype is not None and t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+
+
+def kda_chunk_fwd(q, k, v, log_alpha, beta, S0=None, cu_seqlens=None, out=None, S_final=None,
+                  *, C: int = 64, output_final_state: bool = True, stream=None):
+    """Chunked KDA prefill.
+
+    Fixed-length: q, k, log_alpha [B, T, H, dk]; v [B, T, H, dv]; beta [B, T, H].
+    Varlen: q, k, log_alpha [T, H, dk] ... and ``cu_seqlens`` int32 [N + 1].
+    Returns ``(out, S_final)`` (S_final is None when ``output_final_state`` is
+    False and no buffer was given).
+    """
+    torch = _torch()
+    dt = _dtype_code(q)
+    if cu_seqlens is None:
+        B, T, H, dk = q.shape
+        N = B
+    else:
+        T, H, dk = q.shape
+        N = cu_seqlens.numel() - 1
+        B = N
+    dv = v.shape[-1]
+    for t, n in ((q, "q"), (k, "k"), (v, "v"), (out, "out")):
+        _check(t, n, q.dtype)
+    for t, n in ((log_alpha, "log_alpha"), (beta, "beta"), (S0, "S0"), (S_final, "S_final")):
+        _check(t, n, torch.float32)
+    _check(cu_seqlens, "cu_seqlens", torch.int32)
+    if k.shape != q.shape or log_alpha.shape != q.shape or v.shape[:-1] != q.shape[:-1] \
+            or tuple(beta.shape) != tuple(q.shape[:-1]):
+        raise ValueError("inconsistent q/k/v/log_alpha/beta shapes")
+    if out is None:
+        out = torch.empty(v.shape, dtype=q.dtype, device=q.device)
+    if S_final is None and output_final_state:
+        S_final = torch.empty((N, H, dk, dv), dtype=torch.float32, device=q.device)
+    st = stream if stream is not None else torch.cuda.current_stream(q.device)
+    rc = chunk_fwd_raw(_ptr(q), _ptr(k), _ptr(v), _ptr(log_alpha), _ptr(beta), _ptr(S0),
+                       _ptr(cu_seqlens), _ptr(out), _ptr(S_final), B, T, H, dk, dv, C, dt,
+                       st.cuda_stream)
+    if rc != 0:
+        raise KDAError(rc, "kda_chunk_fwd")
+    return out, S_final
+
+
+def kda_decode_step(q, k, v, log_alpha, beta, S_inout, out=None, *, stream=None):
+    """One decode step for N sequences: q, k, log_alpha [N, H, dk]; v [N, H, dv];
+    beta [N, H]; S_inout [N, H, dk, dv] fp32 (updated in place).  Returns out."""
+    torch = _torch()
+    dt = _dtype_code(q)
+    N, H, dk = q.shape
+    dv = v.shape[-1]
+    for t, n in ((q, "q"), (k, "k"), (v, "v"), (out, "out")):
+        _check(t, n, q.dtype)
+    for t, n in ((log_alpha, "log_alpha"), (beta, "beta"), (S_inout, "S_inout")):
+        _check(t, n, torch.float32)
+    if out is None:
+        out = torch.empty((N, H, dv), dtype=q.dtype, device=q.device)
+    st = stream if stream is not None else torch.cuda.current_stream(q.device)
+    rc = decode_step_raw(_ptr(q), _ptr(k), _ptr(v), _ptr(log_alpha), _ptr(beta), _ptr(S_inout),
+                         _ptr(out), N, H, dk, dv, dt, st.cuda_stream)
+    if rc != 0:
+        raise KDAError(rc, "kda_decode_step")
+    return out

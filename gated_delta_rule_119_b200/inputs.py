@@ -195,3 +195,36 @@ def make_decode_step(N: int, H: int, dk: int, dv: int, dtype: str, seed, step: i
                      log_alpha=log_alpha, beta=beta, S0=None, cu_seqlens=None,
                      B=N, T=1, H=H, dk=dk, dv=dv, dtype=dtype,
                      meta=dict(seed=seed, step=step, gates=gates))
+
+
+def storage_to_torch(x: np.ndarray, dtype: str, device="cpu", pin: bool = False):
+    """A stored array as a torch tensor of the matching dtype (bf16 bits are
+    reinterpreted, not converted)."""
+    import torch
+    if dtype == "bf16" and x.dtype == np.uint16:
+        t = torch.from_numpy(np.ascontiguousarray(x).view(np.int16)).view(torch.bfloat16)
+    else:
+        t = torch.from_numpy(np.ascontiguousarray(x))
+    if pin:
+        t = t.pin_memory()
+    return t.to(device) if device != "cpu" else t
+
+
+def to_torch(inp: KDAInputs, device="cuda", pin: bool = False) -> dict:
+    """Upload one batch: returns q, k, v, log_alpha, beta, S0, cu_seqlens tensors.
+    Fixed-length prefill batches get the [B, T, H, d] view; varlen batches and
+    decode steps stay packed ([T_total, H, d] and [N, H, d])."""
+    import torch
+    d = {}
+    for name in ("q", "k", "v"):
+        d[name] = storage_to_torch(getattr(inp, name), inp.dtype, device, pin)
+    d["log_alpha"] = storage_to_torch(inp.log_alpha, "f32", device, pin)
+    d["beta"] = storage_to_torch(inp.beta, "f32", device, pin)
+    d["S0"] = None if inp.S0 is None else storage_to_torch(inp.S0, "f32", device, pin)
+    d["cu_seqlens"] = None if inp.cu_seqlens is None else \
+        storage_to_torch(inp.cu_seqlens.astype(np.int32), "f32", device, pin)
+    if inp.cu_seqlens is None and "step" not in inp.meta:
+        for name in ("q", "k", "v", "log_alpha", "beta"):
+            t = d[name]
+            d[name] = t.view(inp.B, inp.T, *t.shape[1:])
+    return d

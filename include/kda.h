@@ -1,0 +1,124 @@
+/*
+ * kda.h -- C ABI of libkda.so: Kimi Delta Attention (KDA) on NVIDIA B200 (sm_100a).
+ *
+ * KDA is the gated delta-rule sequence mixer.  For one sequence and one head,
+ * with a d_k x d_v fp32 state S, per token t:
+ *
+ *   S_t = (I - beta_t k_t k_t^T) Diag(alpha_t) S_{t-1} + beta_t k_t v_t^T
+ *   o_t = S_t^T (s q_t),   s = d_k^{-1/2},   alpha_t = exp(log_alpha_t) per channel
+ *
+ * Definition: page "会加减乘除就够:十个问题,手算读懂 Kimi K3 心脏里的全部数学"
+ * (jokeuncle.github.io), intro and 终局 (the four actions forget / correct / write /
+ * read of Q3, Q4, Q6, Q8); the query scale d_k^{-1/2} is the one of the translated
+ * KDA bra-ket blog (mynewscn.com), preamble.  The chunked algorithm used by
+ * kda_chunk_fwd is the WY/UT form of page "22,580：从 GPT-2 到 Kimi K3" §6.3
+ * (yichencityu.github.io), with the per-channel cumulative decay of its §08/§9.1.
+ * Chunking changes only the rounding, never the result.
+ *
+ * Conventions for every entry point:
+ *  - All tensor arguments are DEVICE pointers on the current CUDA device, row-major,
+ *    contiguous, 16-byte aligned.  The caller allocates and owns every buffer; the
+ *    library keeps no pointer after a call returns and allocates no device memory.
+ *  - Calls are asynchronous on `stream` (a cudaStream_t; NULL = legacy default
+ *    stream) and never synchronise the device.
+ *  - The return value is KDA_OK (0) or a negative kda_status.  Argument errors are
+ *    detected on the host before anything is launched; nothing is written then.
+ *  - Input domain: log_alpha finite and <= 0 (alpha in (0, 1]); beta in [0, 1];
+ *    keys are expected to be L2-normalised (not checked).  NaN/Inf inputs give
+ *    unspecified values but never an out-of-bounds access.
+ *  - Thread safety: entry points may be called concurrently from several host
+ *    threads; kda_status_string's CUDA message is kept per host thread.
+ */
+#ifndef KDA_H
+#define KDA_H
+
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* A cudaStream_t, declared without the CUDA headers. */
+typedef struct CUstream_st *kda_stream_t;
+
+/* Element type of q, k, v and out.  log_alpha, beta and the state are always fp32. */
+enum kda_dtype {
+    KDA_F32 = 0,  /* fp32 inputs and outputs; fp32 SIMT arithmetic */
+    KDA_BF16 = 1  /* bf16 inputs and outputs; bf16 tensor-core products, fp32 accumulation and state */
+};
+
+enum kda_status {
+    KDA_OK = 0,
+    KDA_ERR_NULL = -1,    /* a required pointer is NULL */
+    KDA_ERR_DIM = -2,     /* a size is out of range: B, H < 1, T < 0, dk or dv not in {32, 64, 128},
+                             or a combination the dtype does not support */
+    KDA_ERR_CHUNK = -3,   /* C != 64 */
+    KDA_ERR_ALIGN = -4,   /* a pointer is not 16-byte aligned */
+    KDA_ERR_DTYPE = -5,   /* dtype is not a kda_dtype */
+    KDA_ERR_ALIAS = -6,   /* an output overlaps an input it must not overlap */
+    KDA_ERR_CUDA = -7,    /* a CUDA launch failed; kda_status_string names the CUDA error */
+    KDA_ERR_TIMEOUT = -8  /* reserved for bounded device-side waits */
+};
+
+/*
+ * kda_chunk_fwd -- chunked prefill over whole sequences.
+ *
+ * Layout (T_total = B*T without cu_seqlens, T with it):
+ *   q, k       [T_total, H, dk]   dtype            (B x T x H x dk when fixed-length)
+ *   v          [T_total, H, dv]   dtype
+ *   log_alpha  [T_total, H, dk]   fp32             per-channel log-decay, <= 0
+ *   beta       [T_total, H]       fp32             write strength
+ *   S0         [N, H, dk, dv]     fp32 or NULL     initial state (NULL = zero state)
+ *   cu_seqlens [N + 1]            int32 or NULL    NULL: N = B sequences of T tokens each.
+ *                                                 Else N = B sequences packed on the token
+ *                                                 axis: sequence n is tokens
+ *                                                 [cu_seqlens[n], cu_seqlens[n+1]); entries
+ *                                                 must be non-decreasing from 0 to T.  They are
+ *                                                 read on the device and clamped to [0, T], so
+ *                                                 malformed offsets give unspecified values but
+ *                                                 never an out-of-bounds access.
+ *   out        [T_total, H, dv]   dtype            o_t for every token (written)
+ *   S_final    [N, H, dk, dv]     fp32 or NULL     state after each sequence's last token
+ *                                                 (NULL = not written).  May be the same
+ *                                                 pointer as S0 (updated in place).
+ *   C          chunk length; must be 64.
+ * Empty sequences (and T = 0) are allowed: their S_final is S0 (or zero).
+ * Supported sizes: KDA_F32 any dk, dv in {32, 64, 128}; KDA_BF16 dk = dv = 128, or
+ * dk, dv in {32, 64, 128} through the same path.
+ * q, k, v, log_alpha, beta and out may be NULL only when T_total = 0.
+ * Errors: KDA_ERR_NULL (q, k, v, log_alpha, beta or out NULL while T_total > 0), KDA_ERR_DIM, KDA_ERR_CHUNK,
+ * KDA_ERR_DTYPE, KDA_ERR_ALIGN, KDA_ERR_ALIAS (out overlapping an input; S_final
+ * overlapping an input other than exactly S0), KDA_ERR_CUDA.
+ */
+int kda_chunk_fwd(const void *q, const void *k, const void *v, const float *log_alpha,
+                  const float *beta, const float *S0, const int32_t *cu_seqlens, void *out,
+                  float *S_final, int B, int T, int H, int dk, int dv, int C, int dtype,
+                  kda_stream_t stream);
+
+/*
+ * kda_decode_step -- one recurrent step (one new token) for N independent sequences.
+ * The recurrence of the definition above, applied once: forget, look up, correct,
+ * write, read ("Ten questions" Q3-Q8; the token loop of "22,580" §6.1).
+ *   q, k       [N, H, dk]        dtype
+ *   v          [N, H, dv]        dtype
+ *   log_alpha  [N, H, dk]        fp32
+ *   beta       [N, H]            fp32
+ *   S_inout    [N, H, dk, dv]    fp32   state, read and overwritten in place
+ *   out        [N, H, dv]        dtype  o for the new token
+ * Errors: KDA_ERR_NULL, KDA_ERR_DIM (N, H < 1; dk, dv not in {32, 64, 128}),
+ * KDA_ERR_DTYPE, KDA_ERR_ALIGN, KDA_ERR_ALIAS (out or S_inout overlapping an input
+ * or each other), KDA_ERR_CUDA.
+ */
+int kda_decode_step(const void *q, const void *k, const void *v, const float *log_alpha,
+                    const float *beta, float *S_inout, void *out, int N, int H, int dk,
+                    int dv, int dtype, kda_stream_t stream);
+
+/* A static, human-readable description of a status code.  For KDA_ERR_CUDA it names
+ * the CUDA error of the calling host thread's last failed launch. */
+const char *kda_status_string(int status);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* KDA_H */

@@ -1,0 +1,231 @@
+"""GPU parity: libkda.so (through its C ABI) against the fp64 oracle.
+
+Error metric, per output tensor: max|x - r| / max|r| (l-infinity relative over
+the whole tensor), for o and for the final state.  Bars: 1e-4 for fp32 inputs,
+2e-2 for bf16 inputs.  Inputs are the seeded synthetic ones of
+``gated_delta_rule_119_b200.inputs``; the oracle reads the same bytes.
+"""
+import numpy as np
+import pytest
+
+import oracle
+from gated_delta_rule_119_b200.inputs import (WORKLOADS, make_decode_state, make_decode_step,
+                                             make_inputs, make_workload, to_torch)
+
+torch = pytest.importorskip("torch")
+pytestmark = pytest.mark.gpu
+TOL = {"f32": 1e-4, "bf16": 2e-2}
+
+
+def rel_err(x, r):
+    return float(np.abs(x - r).max() / max(np.abs(r).max(), 1e-30))
+
+
+def kda():
+    from gated_delta_rule_119_b200 import kda_chunk_fwd, kda_decode_step
+    return kda_chunk_fwd, kda_decode_step
+
+
+def run_chunk(inp, S_final=True):
+    chunk_fwd, _ = kda()
+    d = to_torch(inp)
+    out, Sf = chunk_fwd(d["q"], d["k"], d["v"], d["log_alpha"], d["beta"], d["S0"],
+                        d["cu_seqlens"], output_final_state=S_final)
+    torch.cuda.synchronize()
+    o = out.float().cpu().numpy().reshape(inp.total_tokens, inp.H, inp.dv)
+    return o, (None if Sf is None else Sf.cpu().numpy())
+
+
+def check_against_oracle(inp, tol=None, tasks=None):
+    tol = TOL[inp.dtype] if tol is None else tol
+    o, S = run_chunk(inp)
+    cu = inp.offsets()
+    if tasks is None:
+        ro, rS = oracle.recurrent_full(inp.q, inp.k, inp.v, inp.log_alpha, inp.beta, inp.S0, cu)
+        eo, es = rel_err(o, ro), rel_err(S, rS)
+    else:
+        outs, sts = oracle.recurrent(inp.q, inp.k, inp.v, inp.log_alpha, inp.beta, inp.S0, cu,
+                                     tasks=tasks)
+        go = np.concatenate([o[cu[n]:cu[n + 1], h].ravel() for n, h in tasks])
+        ro = np.concatenate([x.ravel() for x in outs])
+        eo = rel_err(go, ro)
+        es = max(rel_err(S[n, h], s) for (n, h), s in zip(tasks, sts))
+    assert eo <= tol, f"o: max rel err {eo:.3e} > {tol}"
+    assert es <= tol, f"S_final: max rel err {es:.3e} > {tol}"
+    return eo, es
+
+
+# ------------------------------------------------------------------ small cases
+def test_tiny_f32_workload():
+    """The fp32 workload (B=1, H=2, T=128, dk=dv=32, S0=0) in full."""
+    check_against_oracle(make_workload("tiny_f32"))
+
+
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+@pytest.mark.parametrize("T", [1, 2, 63, 64, 65, 130])
+@pytest.mark.parametrize("d", [32, 128])
+def test_small_shapes(dtype, T, d):
+    check_against_oracle(make_inputs(2, T, 3, d, d, dtype, 100 + T + d, state=T % 2 == 1))
+
+
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+@pytest.mark.parametrize("dk,dv", [(64, 128), (128, 64), (32, 64), (64, 64)])
+def test_rectangular_heads(dtype, dk, dv):
+    check_against_oracle(make_inputs(2, 150, 2, dk, dv, dtype, 7 + dk + dv, state=True))
+
+
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+def test_varlen_ragged_with_empty_sequences(dtype):
+    cu = [0, 0, 1, 65, 65, 200, 263, 263]
+    check_against_oracle(make_inputs(7, 0, 3, 128, 128, dtype, 211, state=True, cu_seqlens=cu))
+
+
+def test_zero_tokens_returns_initial_state():
+    inp = make_inputs(3, 0, 2, 64, 64, "bf16", 5, state=True, cu_seqlens=[0, 0, 0, 0])
+    chunk_fwd, _ = kda()
+    d = to_torch(inp)
+    out, Sf = chunk_fwd(d["q"], d["k"], d["v"], d["log_alpha"], d["beta"], d["S0"],
+                        d["cu_seqlens"])
+    torch.cuda.synchronize()
+    np.testing.assert_array_equal(Sf.cpu().numpy(), inp.S0)
+
+
+def test_final_state_optional_and_in_place():
+    inp = make_inputs(2, 100, 2, 128, 128, "bf16", 9, state=True)
+    chunk_fwd, _ = kda()
+    d = to_torch(inp)
+    o1, _ = chunk_fwd(d["q"], d["k"], d["v"], d["log_alpha"], d["beta"], d["S0"],
+                      output_final_state=False)
+    S = d["S0"].clone()
+    o2, S2 = chunk_fwd(d["q"], d["k"], d["v"], d["log_alpha"], d["beta"], S, S_final=S)
+    torch.cuda.synchronize()
+    assert S2.data_ptr() == S.data_ptr()
+    _, ref = run_chunk(inp)
+    np.testing.assert_array_equal(o1.cpu().float().numpy(), o2.cpu().float().numpy())
+    np.testing.assert_array_equal(S.cpu().numpy(), ref)
+
+
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+def test_degenerate_gates(dtype):
+    """alpha -> 0 (log_alpha = -1e4: the memory is cleared every token), beta = 0
+    (nothing written), beta = 1, and no forgetting, mixed across heads."""
+    inp = make_inputs(2, 140, 4, 128, 128, dtype, 17, state=True)
+    inp.log_alpha[:, 0] = -1e4
+    inp.beta[:, 1] = 0.0
+    inp.beta[:, 2] = 1.0
+    inp.log_alpha[:, 3] = 0.0
+    inp.log_alpha[::7, 2] = -1e4
+    check_against_oracle(inp)
+
+
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+def test_extreme_gates_small(dtype):
+    check_against_oracle(make_inputs(2, 300, 4, 128, 128, dtype, 19, gates="extremes",
+                                     state=True))
+
+
+# ---------------------------------------------------------- full-size workloads
+def sampled_tasks(inp, k, seed):
+    rng = np.random.default_rng(seed)
+    n_seq = inp.n_seqs
+    lens = np.diff(inp.offsets())
+    tasks = {(int(np.argmax(lens)), int(rng.integers(inp.H)))}      # the longest sequence
+    while len(tasks) < k:
+        tasks.add((int(rng.integers(n_seq)), int(rng.integers(inp.H))))
+    return sorted(tasks)
+
+
+@pytest.mark.parametrize("name", ["prefill", "varlen", "extremes"])
+def test_full_workload_sampled(name):
+    """Each bf16 prefill workload at its full size, in the launch configuration the
+    bench times; the oracle recomputes a sample of whole (sequence, head) pairs."""
+    inp = make_workload(name)
+    tasks = sampled_tasks(inp, 6, 1234)
+    if name == "extremes":       # both gate regimes
+        tasks = sorted(set(tasks) | {(0, 0), (3, inp.H - 1)})
+    check_against_oracle(inp, tasks=tasks)
+
+
+# ----------------------------------------------------------------------- decode
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+@pytest.mark.parametrize("dk,dv", [(128, 128), (32, 32), (64, 128), (128, 64)])
+def test_decode_steps(dtype, dk, dv):
+    _, decode = kda()
+    N, H, steps = 5, 3, 6
+    S0 = make_decode_state(N, H, dk, dv, 77)
+    S = torch.from_numpy(S0).cuda()
+    ins = [make_decode_step(N, H, dk, dv, dtype, 77, t) for t in range(steps)]
+    outs = []
+    for inp in ins:
+        d = to_torch(inp)
+        outs.append(decode(d["q"], d["k"], d["v"], d["log_alpha"], d["beta"], S).float()
+                    .cpu().numpy())
+    torch.cuda.synchronize()
+    # oracle: each sequence is a run of `steps` tokens
+    cat = lambda name: np.stack([getattr(i, name) for i in ins], axis=1).reshape(
+        N * steps, *getattr(ins[0], name).shape[1:])
+    cu = np.arange(N + 1) * steps
+    ro, rS = oracle.recurrent_full(cat("q"), cat("k"), cat("v"), cat("log_alpha"), cat("beta"),
+                                   S0, cu)
+    go = np.stack(outs, axis=1).reshape(N * steps, H, dv)
+    tol = TOL[dtype]
+    assert rel_err(go, ro) <= tol
+    assert rel_err(S.cpu().numpy(), rS) <= tol
+
+
+def test_decode_workload_sampled():
+    """The decode workload's full state (256 sequences x 32 heads x 128 x 128 fp32),
+    a few steps; the oracle recomputes sampled (sequence, head) pairs."""
+    _, decode = kda()
+    w = WORKLOADS["decode"]
+    N, H, dk, dv, steps = w["B"], w["H"], w["dk"], w["dv"], 4
+    S0 = make_decode_state(N, H, dk, dv, w["index"])
+    S = torch.from_numpy(S0).cuda()
+    ins = [make_decode_step(N, H, dk, dv, "bf16", w["index"], t) for t in range(steps)]
+    outs = []
+    for inp in ins:
+        d = to_torch(inp)
+        outs.append(decode(d["q"], d["k"], d["v"], d["log_alpha"], d["beta"], S).float()
+                    .cpu().numpy())
+    Sg = S.cpu().numpy()
+    rng = np.random.default_rng(3)
+    for n, h in zip(rng.integers(N, size=6), rng.integers(H, size=6)):
+        pick = lambda name: np.stack([getattr(i, name)[n, h] for i in ins])[:, None]
+        ro, rS = oracle.recurrent_full(pick("q"), pick("k"), pick("v"), pick("log_alpha"),
+                                       pick("beta"), S0[n:n + 1, h:h + 1].copy())
+        assert rel_err(np.stack([o[n, h] for o in outs]), ro[:, 0]) <= TOL["bf16"]
+        assert rel_err(Sg[n, h], rS[0, 0]) <= TOL["bf16"]
+
+
+def test_decode_matches_prefill():
+    """T decode steps == one prefill over the same T tokens (both on the GPU)."""
+    chunk_fwd, decode = kda()
+    inp = make_inputs(3, 70, 2, 128, 128, "bf16", 31, state=True)
+    o_pre, S_pre = run_chunk(inp)
+    d = to_torch(inp)
+    S = d["S0"].clone()
+    outs = []
+    for t in range(inp.T):
+        outs.append(decode(d["q"][:, t].contiguous(), d["k"][:, t].contiguous(),
+                           d["v"][:, t].contiguous(), d["log_alpha"][:, t].contiguous(),
+                           d["beta"][:, t].contiguous(), S))
+    o_dec = torch.stack(outs, 1).float().cpu().numpy().reshape(-1, inp.H, inp.dv)
+    assert rel_err(o_dec, o_pre) <= TOL["bf16"]
+    assert rel_err(S.cpu().numpy(), S_pre) <= TOL["bf16"]
+
+
+# ------------------------------------------------------ errors with real memory
+def test_errors_with_device_tensors():
+    from gated_delta_rule_119_b200 import KDAError
+    chunk_fwd, decode = kda()
+    inp = make_inputs(1, 64, 1, 128, 128, "bf16", 3)
+    d = to_torch(inp)
+    with pytest.raises(KDAError, match="KDA_ERR_ALIAS"):
+        chunk_fwd(d["q"], d["k"], d["v"], d["log_alpha"], d["beta"], out=d["v"])
+    raw = torch.empty(64 * 128 + 1, dtype=torch.bfloat16, device="cuda")
+    qm = raw[1:].view(1, 64, 1, 128)                      # 2-byte offset: misaligned
+    qm.copy_(d["q"])
+    with pytest.raises(KDAError, match="KDA_ERR_ALIGN"):
+        chunk_fwd(qm, d["k"], d["v"], d["log_alpha"], d["beta"])
+    with pytest.raises(KDAError, match="KDA_ERR_CHUNK"):
+        chunk_fwd(d["q"], d["k"], d["v"], d["log_alpha"], d["beta"], C=128)
