@@ -295,7 +295,8 @@ def run_ours(args, rank, local_rank, world):
         bytes_per_launch = alg_bytes_prefill(tok_heads, inp.n_seqs * inp.H, inp.dk, inp.dv, es,
                                              inp.S0 is not None, True)
         flops_per_launch = alg_flops_prefill(tok_heads, inp.dk, inp.dv)
-        kernel_key = "chunk_simt"
+        kernel_key = "chunk" if (w["dtype"] == "bf16" and w["dk"] == 128 and w["dv"] == 128) \
+            else "chunk_simt"
         inp_for_cpu = inp
 
     for i in range(args.warmup):

@@ -16,7 +16,7 @@ KDA_F32, KDA_BF16 = 0, 1
 STATUS = {0: "KDA_OK", -1: "KDA_ERR_NULL", -2: "KDA_ERR_DIM", -3: "KDA_ERR_CHUNK",
           -4: "KDA_ERR_ALIGN", -5: "KDA_ERR_DTYPE", -6: "KDA_ERR_ALIAS", -7: "KDA_ERR_CUDA",
           -8: "KDA_ERR_TIMEOUT"}
-EXPORTS = ("kda_chunk_fwd", "kda_decode_step", "kda_status_string")
+EXPORTS = ("kda_chunk_fwd", "kda_decode_step", "kda_device_status", "kda_status_string")
 
 _lib = None
 
@@ -42,11 +42,19 @@ def load_library(path: str | None = None):
     lib.kda_chunk_fwd.restype = ctypes.c_int
     lib.kda_decode_step.argtypes = [V, V, V, F, F, F, V] + [I32] * 5 + [V]
     lib.kda_decode_step.restype = ctypes.c_int
+    lib.kda_device_status.argtypes = []
+    lib.kda_device_status.restype = ctypes.c_int
     lib.kda_status_string.argtypes = [ctypes.c_int]
     lib.kda_status_string.restype = ctypes.c_char_p
     if path is None:
         _lib = lib
     return lib
+
+
+def kda_device_status() -> int:
+    """Synchronise the device; KDA_ERR_TIMEOUT (-8) if a kernel gave up a bounded
+    wait since the previous call, else 0.  Clears the record."""
+    return load_library().kda_device_status()
 
 
 def kda_status_string(status: int) -> str:

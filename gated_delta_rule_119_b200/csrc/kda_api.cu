@@ -102,3 +102,10 @@ extern "C" int kda_decode_step(const void *q, const void *k, const void *v, cons
     KdaDecodeArgs a{q, k, v, log_alpha, beta, S_inout, out, N, H, dk, dv, 1.0f / sqrtf((float)dk)};
     return cuda_status(kda_launch_decode(a, dtype, reinterpret_cast<cudaStream_t>(stream)));
 }
+
+extern "C" int kda_device_status(void) {
+    unsigned int st = 0;
+    const cudaError_t e = kda_read_device_status(&st, true);
+    if (e != cudaSuccess) return cuda_status(e);
+    return st ? KDA_ERR_TIMEOUT : KDA_OK;
+}

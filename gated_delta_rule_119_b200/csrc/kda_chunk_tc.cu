@@ -1,5 +1,543 @@
-// Tensor-core (tcgen05) chunk path: placeholder until the kernel lands.
-#include "kda_common.cuh"
+// Chunked KDA prefill on the sm_100a tensor cores (bf16 q/k/v, dk = dv = 128, C = 64).
+//
+// One CTA owns one (sequence, head, 64-column slice of d_v) and walks the
+// sequence chunk by chunk, carrying the fp32 state slice S (128 x 64) in
+// tensor memory.  Chunk algebra ("22,580" §6.3 WY/UT form with the per-channel
+// cumulative decay of its §08/§9.1; all decay factors are products of alphas
+// over the steps strictly after the write up to the read):
+//
+//   A[r][i]  = beta_r sum_c k_rc k_ic D_ric  (i < r),   P[r][i] = s sum_c q_rc k_ic D_ric  (i <= r)
+//   T'       = (I + A)^{-1} Diag(beta)
+//   W        = T' (k gamma),  u = T' v - W S,  o = (s q gamma) S + P u
+//   S       <- Diag(gamma_last) S + (k kappa)^T u
+//
+// The output is computed from S without waiting for u:
+//   o = (s q gamma - P W) S + (P T') v,
+// so one tensor-core accumulation produces both u (rows 0-63) and o (rows
+// 64-127):  [u; o] = [T'; P T'] v + [-W; s q gamma - P W] S.
+//
+// Per chunk:
+//  E1  stage q, k (row-major) and the v slice (swizzled) in shared memory.
+//  E2  one thread per (channel, pair of 16-row blocks): alpha = exp(log_alpha),
+//      block-local running products, and from them the operands k gamma,
+//      k kappa (tensor-core layout) and the factored operands of the 16 x 16
+//      blocks of A and P.  A block (a, b) of A is (k f)_a (k h)_b^T times a
+//      per-channel scale, where f, h are block-local products rescaled by
+//      rho = exp(-sum_block log_alpha / 2) so that every factor stays in
+//      [e^-70, e^70].  A diagonal block whose decay spread exceeds that range
+//      is handled per channel by exact running products instead.
+//  AP  A and P from those factors with warp-level bf16 MMAs (fp32 accumulation).
+//  T   T = (I + A)^{-1} by blocked forward substitution in fp32; T', P T'.
+//  TC  tcgen05: [W; P W] = [T'; P T'] (k gamma); state readout (bf16 copy,
+//      decay in place); [u; o] as above; S += (k kappa)^T u.
+#include <stdio.h>
 
-bool kda_chunk_tc_supports(int, int) { return false; }
-cudaError_t kda_launch_chunk_tc(const KdaChunkArgs &, cudaStream_t) { return cudaErrorNotSupported; }
+#include "kda_common.cuh"
+#include "kda_tc_util.cuh"
+
+__device__ unsigned int g_kda_device_status = 0;
+
+namespace {
+using namespace kda_tc;
+
+constexpr int CH = 64, DK = 128, DV = 128;
+constexpr int DVT = 64;                 // d_v columns per CTA
+constexpr int NTILE = DV / DVT;         // CTAs per (sequence, head)
+constexpr int NTHR = 256;
+constexpr int LP = 136;                 // row pitch (bf16) of the warp-MMA operand tiles
+constexpr int LF = 68;                  // row pitch (fp32) of the 64 x 64 matrices
+constexpr float kSpreadLimit = 140.f;   // -sum log_alpha over 16 rows beyond which a block is exact-path
+constexpr long long kWaitCycles = 4000000000LL;   // about 2 s at B200 clocks
+constexpr uint32_t kTmemCols = 256;
+
+// Shared-memory map (bytes from a 1024-byte aligned base).
+constexpr uint32_t OFF_V = 0;                       // v slice, then u: 64 lines (MN-major B)
+constexpr uint32_t OFF_TP = OFF_V + 8192;           // [T'; P T']: 128 lines (K-major A)
+constexpr uint32_t OFF_KT = OFF_TP + 16384;         // k gamma: 2 x 64 lines (MN-major B)
+constexpr uint32_t OFF_KC = OFF_KT + 16384;         // k kappa: 2 x 64 lines (MN-major A)
+constexpr uint32_t OFF_X = OFF_KC + 16384;          // region X, reused:
+constexpr uint32_t X_KL = 0, X_KR = 17408, X_TM = 34816, X_QL = 52224, X_SIZE = 69632;
+constexpr uint32_t X_A2 = 0, X_S = 32768;           //   later [-W; Q'] (2 x 128 lines) and S (128 lines)
+constexpr uint32_t OFF_Q = OFF_X + X_SIZE;          // raw q [64][128] bf16
+constexpr uint32_t OFF_K = OFF_Q + 16384;           // raw k
+constexpr uint32_t OFF_AM = OFF_K + 16384;          // A [64][LF] fp32
+constexpr uint32_t OFF_PM = OFF_AM + 17408;         // P [64][LF] fp32
+constexpr uint32_t OFF_SMALL = OFF_PM + 17408;
+constexpr uint32_t SM_BETA = OFF_SMALL;             // [64]
+constexpr uint32_t SM_GC = SM_BETA + 256;           // [128]   gamma_last
+constexpr uint32_t SM_BS = SM_GC + 512;             // [4][128] sum of log_alpha per block
+constexpr uint32_t SM_BT = SM_BS + 2048;            // [4][128] product of alpha per block
+constexpr uint32_t SM_SC = SM_BT + 2048;            // [10][128] per-channel scale of block (a, b)
+constexpr uint32_t SM_QF = SM_SC + 5120;            // [4][128] (s q f) -> s q gamma factor
+constexpr uint32_t SM_XT = SM_QF + 2048;            // [3][16][16] forward-substitution scratch
+constexpr uint32_t SM_END = SM_XT + 3072;
+constexpr size_t kSmemBytes = SM_END + 1024;        // + alignment slack
+static_assert(OFF_X % 1024 == 0 && (OFF_X + X_S) % 1024 == 0, "tile alignment");
+static_assert(X_S + 16384 <= X_QL, "S copy must not reach the q operand");
+static_assert(kSmemBytes <= 232448, "shared memory budget");
+
+__constant__ int kPairA[10] = {0, 1, 1, 2, 2, 2, 3, 3, 3, 3};
+__constant__ int kPairB[10] = {0, 0, 1, 0, 1, 2, 0, 1, 2, 3};
+
+__device__ __forceinline__ float bf(const __nv_bfloat16 *p) { return __bfloat162float(*p); }
+
+__global__ void __launch_bounds__(NTHR, 1) kda_chunk_tc_kernel(KdaChunkArgs a) {
+    extern __shared__ uint8_t smraw[];
+    uint8_t *sm = (uint8_t *)(((uintptr_t)smraw + 1023) & ~(uintptr_t)1023);
+    __shared__ uint64_t bar_w, bar_uo, bar_s;
+    __shared__ uint32_t s_tmem;
+    __shared__ int s_abort;
+
+    uint8_t *sV = sm + OFF_V, *sTP = sm + OFF_TP, *sKt = sm + OFF_KT, *sKC = sm + OFF_KC;
+    uint8_t *sX = sm + OFF_X;
+    __nv_bfloat16 *KL = (__nv_bfloat16 *)(sX + X_KL), *KR = (__nv_bfloat16 *)(sX + X_KR);
+    __nv_bfloat16 *QL = (__nv_bfloat16 *)(sX + X_QL);
+    float *Tm = (float *)(sX + X_TM);
+    uint8_t *sA2 = sX + X_A2, *sS = sX + X_S;
+    const __nv_bfloat16 *sQ = (const __nv_bfloat16 *)(sm + OFF_Q);
+    const __nv_bfloat16 *sK = (const __nv_bfloat16 *)(sm + OFF_K);
+    float *Am = (float *)(sm + OFF_AM), *Pm = (float *)(sm + OFF_PM);
+    float *sBeta = (float *)(sm + SM_BETA), *sGC = (float *)(sm + SM_GC);
+    float *sBS = (float *)(sm + SM_BS), *sBT = (float *)(sm + SM_BT);
+    float *sSC = (float *)(sm + SM_SC), *sQF = (float *)(sm + SM_QF), *sXT = (float *)(sm + SM_XT);
+
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int H = a.H;
+    const int pair = blockIdx.x / NTILE, tile = blockIdx.x % NTILE;
+    const int n = pair / H, h = pair % H;
+    const float scale = a.scale;
+    const __nv_bfloat16 *qg = static_cast<const __nv_bfloat16 *>(a.q);
+    const __nv_bfloat16 *kg = static_cast<const __nv_bfloat16 *>(a.k);
+    const __nv_bfloat16 *vg = static_cast<const __nv_bfloat16 *>(a.v);
+    __nv_bfloat16 *og = static_cast<__nv_bfloat16 *>(a.out);
+    int64_t t0, t1;
+    kda::seq_bounds(a.cu_seqlens, n, a.T, a.T_total, t0, t1);
+
+    if (tid == 0) {
+        mbar_init(&bar_w, 1);
+        mbar_init(&bar_uo, 1);
+        mbar_init(&bar_s, 1);
+        mbar_init_fence();
+        s_abort = 0;
+    }
+    if (warp == 0) tmem_alloc(&s_tmem, kTmemCols);
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = s_tmem;
+    const uint32_t T_S = tmem, T_UO = tmem + DVT, T_W = tmem + 2 * DVT;
+    const int quarter = warp & 3, half = warp >> 2;
+    const uint32_t lane_off = (uint32_t)(32 * quarter) << 16;
+    const int trow = 32 * quarter + lane;       // the TMEM lane (matrix row) this thread serves
+    const size_t s_base = ((size_t)pair * DK) * DV + (size_t)tile * DVT + half * 32;
+
+    {   // initial state slice -> TMEM
+        float v[32];
+        if (a.S0) {
+            const float4 *src = reinterpret_cast<const float4 *>(a.S0 + s_base + (size_t)trow * DV);
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+                const float4 x = src[i];
+                v[4 * i] = x.x; v[4 * i + 1] = x.y; v[4 * i + 2] = x.z; v[4 * i + 3] = x.w;
+            }
+        } else {
+#pragma unroll
+            for (int i = 0; i < 32; ++i) v[i] = 0.f;
+        }
+        tmem_st32(T_S + lane_off + half * 32, v);
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+
+    const int nchunks = (int)((t1 - t0 + CH - 1) / CH);
+    uint64_t *pending = nullptr;
+    uint32_t pending_par = 0;
+    for (int ci = 0; ci < nchunks; ++ci) {
+        const uint32_t par = (uint32_t)(ci & 1);
+        const int64_t c0 = t0 + (int64_t)ci * CH;
+        const int nr = (int)(t1 - c0 < CH ? t1 - c0 : CH);
+
+        // ---------------- E1: stage q, k, v slice, beta; clear the diagonal blocks of A, P
+        for (int idx = tid; idx < 2048; idx += NTHR) {
+            const int which = idx >> 10, rem = idx & 1023, r = rem >> 4, j = rem & 15;
+            const int rs = r < nr ? r : nr - 1;
+            const __nv_bfloat16 *src = (which ? kg : qg) + ((size_t)(c0 + rs) * H + h) * DK + j * 8;
+            cp_async16(sm + (which ? OFF_K : OFF_Q) + r * 256 + j * 16, src, r < nr ? 16u : 0u);
+        }
+        for (int idx = tid; idx < 512; idx += NTHR) {
+            const int r = idx >> 3, j = idx & 7;
+            const int rs = r < nr ? r : nr - 1;
+            const __nv_bfloat16 *src = vg + ((size_t)(c0 + rs) * H + h) * DV + tile * DVT + j * 8;
+            cp_async16(sV + sw128_chunk(r, j), src, r < nr ? 16u : 0u);
+        }
+        if (tid < CH) sBeta[tid] = tid < nr ? a.beta[(size_t)(c0 + tid) * H + h] : 0.f;
+        for (int idx = tid; idx < 2048; idx += NTHR) {
+            const int m = idx >> 10, rem = idx & 1023, blk = rem >> 8, r = (rem >> 4) & 15, i = rem & 15;
+            (m ? Pm : Am)[(16 * blk + r) * LF + 16 * blk + i] = 0.f;
+        }
+        cp_async_wait_all();
+        __syncthreads();
+
+        // ---------------- E2 pass 1: alpha, per-block sums and products
+        const int ch = tid & 127, hb = tid >> 7;     // channel, pair of blocks {2hb, 2hb+1}
+        float al[32];
+#pragma unroll
+        for (int rr = 0; rr < 32; ++rr) {
+            const int r = 32 * hb + rr;
+            al[rr] = r < nr ? a.log_alpha[((size_t)(c0 + r) * H + h) * DK + ch] : 0.f;
+        }
+#pragma unroll
+        for (int bb = 0; bb < 2; ++bb) {
+            float s = 0.f, p = 1.f;
+#pragma unroll
+            for (int rr = 0; rr < 16; ++rr) {
+                const float la = al[16 * bb + rr];
+                s += la;
+                const float x = expf(la);
+                al[16 * bb + rr] = x;
+                p *= x;
+            }
+            sBS[(2 * hb + bb) * 128 + ch] = s;
+            sBT[(2 * hb + bb) * 128 + ch] = p;
+        }
+        __syncthreads();
+
+        // ---------------- E2 pass 2: operands
+#pragma unroll
+        for (int bb = 0; bb < 2; ++bb) {
+            const int b = 2 * hb + bb;
+            float gpre = 1.f, ksuf = 1.f;
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+                if (j < b) gpre *= sBT[j * 128 + ch];
+                if (j > b) ksuf *= sBT[j * 128 + ch];
+            }
+            const float bs = sBS[b * 128 + ch];
+            const bool flagged = bs < -kSpreadLimit;
+            const float rho = flagged ? 1.f : expf(-0.5f * bs);
+            sQF[b * 128 + ch] = flagged ? gpre : gpre * expf(0.5f * bs);
+            const uint32_t blk_off = (uint32_t)(ch >> 6) * 8192u;
+            float lam = 1.f;
+#pragma unroll
+            for (int rr = 0; rr < 16; ++rr) {
+                const int r = 16 * b + rr;
+                lam *= al[16 * bb + rr];
+                const float kv = bf(&sK[r * 128 + ch]), qv = bf(&sQ[r * 128 + ch]);
+                *(__nv_bfloat16 *)(sKt + blk_off + sw128(r, ch & 63)) = __float2bfloat16_rn(kv * (gpre * lam));
+                KL[r * LP + ch] = __float2bfloat16_rn(kv * (rho * lam));
+                QL[r * LP + ch] = __float2bfloat16_rn(scale * qv * (rho * lam));
+            }
+            float sig = 1.f;
+#pragma unroll
+            for (int rr = 15; rr >= 0; --rr) {
+                const int r = 16 * b + rr;
+                const float kv = bf(&sK[r * 128 + ch]);
+                *(__nv_bfloat16 *)(sKC + blk_off + sw128(r, ch & 63)) = __float2bfloat16_rn(kv * (sig * ksuf));
+                KR[r * LP + ch] = __float2bfloat16_rn(kv * (rho * sig));
+                sig *= al[16 * bb + rr];
+            }
+            if (flagged) {
+                // Exact diagonal-block contribution of this channel (running products).
+#pragma unroll
+                for (int i = 0; i < 16; ++i) {
+                    const float ki = bf(&sK[(16 * b + i) * 128 + ch]);
+                    float f = 1.f;
+#pragma unroll
+                    for (int r = i; r < 16; ++r) {
+                        if (r > i) f *= al[16 * bb + r];
+                        const int R = 16 * b + r, I = 16 * b + i;
+                        const float kd = ki * f;
+                        if (r > i) atomicAdd(&Am[R * LF + I], sBeta[R] * bf(&sK[R * 128 + ch]) * kd);
+                        atomicAdd(&Pm[R * LF + I], scale * bf(&sQ[R * 128 + ch]) * kd);
+                    }
+                }
+            }
+        }
+        if (hb == 0) sGC[ch] = sBT[ch] * sBT[128 + ch] * sBT[256 + ch] * sBT[384 + ch];
+#pragma unroll
+        for (int pp = 0; pp < 5; ++pp) {
+            const int p = 5 * hb + pp, pa = kPairA[p], pb = kPairB[p];
+            float sc;
+            const bool fa = sBS[pa * 128 + ch] < -kSpreadLimit, fb = sBS[pb * 128 + ch] < -kSpreadLimit;
+            if (pa == pb) {
+                sc = fa ? 0.f : 1.f;
+            } else {
+                float e = (fa ? 0.f : 0.5f * sBS[pa * 128 + ch]) + (fb ? 0.f : 0.5f * sBS[pb * 128 + ch]);
+                for (int j = pb + 1; j < pa; ++j) e += sBS[j * 128 + ch];
+                sc = expf(e);
+            }
+            sSC[p * 128 + ch] = sc;
+        }
+        __syncthreads();
+
+        // ---------------- AP: 16 x 16 blocks of A and P with warp MMAs
+        {
+            const int g = lane >> 2, t4 = lane & 3;
+            for (int task = warp; task < 20; task += 8) {
+                const int mat = task / 10, p = task % 10, pa = kPairA[p], pb = kPairB[p];
+                const __nv_bfloat16 *Ls = mat == 0 ? KL : QL;
+                float acc[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+#pragma unroll
+                for (int kt = 0; kt < 8; ++kt) {
+                    const int c = 16 * kt + 2 * t4;
+                    const uint32_t a0 = *(const uint32_t *)&Ls[(16 * pa + g) * LP + c];
+                    const uint32_t a1 = *(const uint32_t *)&Ls[(16 * pa + g + 8) * LP + c];
+                    const uint32_t a2 = *(const uint32_t *)&Ls[(16 * pa + g) * LP + c + 8];
+                    const uint32_t a3 = *(const uint32_t *)&Ls[(16 * pa + g + 8) * LP + c + 8];
+                    const float s0 = sSC[p * 128 + c], s1 = sSC[p * 128 + c + 1];
+                    const float s8 = sSC[p * 128 + c + 8], s9 = sSC[p * 128 + c + 9];
+#pragma unroll
+                    for (int j = 0; j < 2; ++j) {
+                        const int i = 16 * pb + 8 * j + g;
+                        const float2 f0 = unpack_bf16(*(const uint32_t *)&KR[i * LP + c]);
+                        const float2 f1 = unpack_bf16(*(const uint32_t *)&KR[i * LP + c + 8]);
+                        mma_m16n8k16(acc[j], a0, a1, a2, a3, pack_bf16(f0.x * s0, f0.y * s1),
+                                     pack_bf16(f1.x * s8, f1.y * s9));
+                    }
+                }
+#pragma unroll
+                for (int j = 0; j < 2; ++j) {
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        const int r = 16 * pa + g + (e >= 2 ? 8 : 0);
+                        const int i = 16 * pb + 8 * j + 2 * t4 + (e & 1);
+                        const float val = acc[j][e];
+                        if (mat == 0) {
+                            if (pa != pb) Am[r * LF + i] = sBeta[r] * val;
+                            else if (i < r) Am[r * LF + i] += sBeta[r] * val;
+                        } else {
+                            if (pa != pb) Pm[r * LF + i] = val;
+                            else if (i <= r) Pm[r * LF + i] += val;
+                        }
+                    }
+                }
+            }
+        }
+        __syncthreads();
+
+        // ---------------- T = (I + A)^{-1}: diagonal 16 x 16 blocks (one column per lane)
+        if (warp < 4 && lane < 16) {
+            const int w = warp, i = lane;
+            const float *Ab = Am + (16 * w) * LF + 16 * w;
+            float tc[16];
+#pragma unroll
+            for (int r = 0; r < 16; ++r) {
+                float s = r == i ? 1.f : 0.f;
+                if (r > i) {
+                    float acc = 0.f;
+#pragma unroll
+                    for (int m = 0; m < r; ++m)
+                        if (m >= i) acc = fmaf(Ab[r * LF + m], tc[m], acc);
+                    s = -acc;
+                }
+                tc[r] = s;
+            }
+#pragma unroll
+            for (int r = 0; r < 16; ++r) Tm[(16 * w + r) * LF + 16 * w + i] = tc[r];
+        }
+        __syncthreads();
+        //      off-diagonal blocks, by distance d = a - b: T_ab = -T_aa sum_{m=b}^{a-1} A_am T_mb
+        for (int d = 1; d < 4; ++d) {
+            const int nblk = 4 - d;
+            for (int o = tid; o < nblk * 256; o += NTHR) {
+                const int b = o >> 8, pa = b + d, rr = (o >> 4) & 15, ii = o & 15;
+                float x = 0.f;
+                for (int m = b; m < pa; ++m) {
+                    const float *arow = Am + (16 * pa + rr) * LF + 16 * m;
+                    const float *tcol = Tm + (16 * m) * LF + 16 * b + ii;
+#pragma unroll
+                    for (int jj = 0; jj < 16; ++jj) x = fmaf(arow[jj], tcol[jj * LF], x);
+                }
+                sXT[o] = x;
+            }
+            __syncthreads();
+            for (int o = tid; o < nblk * 256; o += NTHR) {
+                const int b = o >> 8, pa = b + d, rr = (o >> 4) & 15, ii = o & 15;
+                const float *trow_ = Tm + (16 * pa + rr) * LF + 16 * pa;
+                const float *xcol = sXT + (b << 8) + ii;
+                float x = 0.f;
+                for (int jj = 0; jj <= rr; ++jj) x = fmaf(trow_[jj], xcol[jj * 16], x);
+                Tm[(16 * pa + rr) * LF + 16 * b + ii] = -x;
+            }
+            __syncthreads();
+        }
+        //      [T'; P T'] -> tensor-core operand (K-major, 128 lines)
+        for (int o = tid; o < CH * CH; o += NTHR) {
+            const int r = o >> 6, i = o & 63;
+            const float tv = i <= r ? Tm[r * LF + i] * sBeta[i] : 0.f;
+            *(__nv_bfloat16 *)(sTP + sw128(r, i)) = __float2bfloat16_rn(tv);
+            float pv = 0.f;
+            for (int m = i; m <= r; ++m) pv = fmaf(Pm[r * LF + m], Tm[m * LF + i], pv);
+            *(__nv_bfloat16 *)(sTP + sw128(64 + r, i)) = __float2bfloat16_rn(i <= r ? pv * sBeta[i] : 0.f);
+        }
+        fence_async_smem();
+        tc_fence_before();
+        __syncthreads();
+        tc_fence_after();
+
+        // ---------------- TC: [W; P W] = [T'; P T'] (k gamma)
+        if (tid == 0) {
+            const uint32_t a0 = smem_u32(sTP), b0 = smem_u32(sKt);
+#pragma unroll
+            for (int ks = 0; ks < 4; ++ks)
+                mma_bf16(T_W, desc_sw128(a0 + 32 * ks, 16, 1024), desc_sw128(b0 + 2048 * ks, 8192, 1024),
+                         idesc_bf16(128, 128, false, true), ks > 0);
+            mma_commit(&bar_w);
+        }
+        //      state slice: bf16 copy for the MMAs, decay in place for the update
+        {
+            float v[32];
+            tmem_ld32(T_S + lane_off + half * 32, v);
+#pragma unroll
+            for (int m = 0; m < 4; ++m) {
+                uint4 pk;
+                pk.x = pack_bf16(v[8 * m + 0], v[8 * m + 1]);
+                pk.y = pack_bf16(v[8 * m + 2], v[8 * m + 3]);
+                pk.z = pack_bf16(v[8 * m + 4], v[8 * m + 5]);
+                pk.w = pack_bf16(v[8 * m + 6], v[8 * m + 7]);
+                *(uint4 *)(sS + sw128_chunk(trow, 4 * half + m)) = pk;
+            }
+            const float gdec = sGC[trow];
+#pragma unroll
+            for (int i = 0; i < 32; ++i) v[i] *= gdec;
+            tmem_st32(T_S + lane_off + half * 32, v);
+        }
+        if (!mbar_wait(&bar_w, par, kWaitCycles)) s_abort = 1;
+        tc_fence_after();
+        //      [-W; s q gamma - P W] -> tensor-core operand (K-major, 2 x 128 lines)
+        {
+#pragma unroll
+            for (int part = 0; part < 2; ++part) {
+                float v[32];
+                tmem_ld32(T_W + lane_off + half * 64 + part * 32, v);
+                const int c0c = half * 64 + part * 32;
+                if (trow >= 64) {
+                    const int r = trow - 64;
+                    const float *qf = sQF + (r >> 4) * 128 + c0c;
+#pragma unroll
+                    for (int i = 0; i < 32; ++i) v[i] = bf(&QL[r * LP + c0c + i]) * qf[i] - v[i];
+                } else {
+#pragma unroll
+                    for (int i = 0; i < 32; ++i) v[i] = -v[i];
+                }
+#pragma unroll
+                for (int m = 0; m < 4; ++m) {
+                    uint4 pk;
+                    pk.x = pack_bf16(v[8 * m + 0], v[8 * m + 1]);
+                    pk.y = pack_bf16(v[8 * m + 2], v[8 * m + 3]);
+                    pk.z = pack_bf16(v[8 * m + 4], v[8 * m + 5]);
+                    pk.w = pack_bf16(v[8 * m + 6], v[8 * m + 7]);
+                    *(uint4 *)(sA2 + half * 16384 + sw128_chunk(trow, 4 * part + m)) = pk;
+                }
+            }
+        }
+        fence_async_smem();
+        tc_fence_before();
+        __syncthreads();
+        if (s_abort) { pending = &bar_w; pending_par = par; break; }
+        tc_fence_after();
+
+        // ---------------- TC: [u; o] = [T'; P T'] v + [-W; Q'] S
+        if (tid == 0) {
+            const uint32_t idesc = idesc_bf16(128, DVT, false, true);
+            const uint32_t tp = smem_u32(sTP), vv = smem_u32(sV), a2 = smem_u32(sA2), ss = smem_u32(sS);
+#pragma unroll
+            for (int ks = 0; ks < 4; ++ks)
+                mma_bf16(T_UO, desc_sw128(tp + 32 * ks, 16, 1024), desc_sw128(vv + 2048 * ks, 8192, 1024),
+                         idesc, ks > 0);
+#pragma unroll
+            for (int ks = 0; ks < 8; ++ks)
+                mma_bf16(T_UO, desc_sw128(a2 + (ks >> 2) * 16384 + 32 * (ks & 3), 16, 1024),
+                         desc_sw128(ss + 2048 * ks, 16384, 1024), idesc, 1);
+            mma_commit(&bar_uo);
+        }
+        if (!mbar_wait(&bar_uo, par, kWaitCycles)) s_abort = 1;
+        tc_fence_after();
+        {
+            float v[32];
+            tmem_ld32(T_UO + lane_off + half * 32, v);
+            uint4 pk[4];
+#pragma unroll
+            for (int m = 0; m < 4; ++m) {
+                pk[m].x = pack_bf16(v[8 * m + 0], v[8 * m + 1]);
+                pk[m].y = pack_bf16(v[8 * m + 2], v[8 * m + 3]);
+                pk[m].z = pack_bf16(v[8 * m + 4], v[8 * m + 5]);
+                pk[m].w = pack_bf16(v[8 * m + 6], v[8 * m + 7]);
+            }
+            if (trow < 64) {
+#pragma unroll
+                for (int m = 0; m < 4; ++m) *(uint4 *)(sV + sw128_chunk(trow, 4 * half + m)) = pk[m];
+            } else if (trow - 64 < nr) {
+                uint4 *dst = reinterpret_cast<uint4 *>(
+                    og + ((size_t)(c0 + trow - 64) * H + h) * DV + tile * DVT + half * 32);
+#pragma unroll
+                for (int m = 0; m < 4; ++m) dst[m] = pk[m];
+            }
+        }
+        fence_async_smem();
+        tc_fence_before();
+        __syncthreads();
+        if (s_abort) { pending = &bar_uo; pending_par = par; break; }
+        tc_fence_after();
+
+        // ---------------- TC: S += (k kappa)^T u
+        if (tid == 0) {
+            const uint32_t kc = smem_u32(sKC), uu = smem_u32(sV);
+#pragma unroll
+            for (int ks = 0; ks < 4; ++ks)
+                mma_bf16(T_S, desc_sw128(kc + 2048 * ks, 8192, 1024), desc_sw128(uu + 2048 * ks, 8192, 1024),
+                         idesc_bf16(128, DVT, true, true), 1);
+            mma_commit(&bar_s);
+        }
+        if (!mbar_wait(&bar_s, par, kWaitCycles)) s_abort = 1;
+        tc_fence_after();
+        __syncthreads();
+        if (s_abort) { pending = &bar_s; pending_par = par; break; }
+    }
+
+    if (pending) {
+        // A tensor-core wait gave up: record it, give the in-flight work one more
+        // bounded wait, and leave without writing the state.
+        if (tid == 0) atomicOr(&g_kda_device_status, 1u);
+        mbar_wait(pending, pending_par, kWaitCycles);
+    } else if (a.S_final) {
+        float v[32];
+        tmem_ld32(T_S + lane_off + half * 32, v);
+        float4 *dst = reinterpret_cast<float4 *>(a.S_final + s_base + (size_t)trow * DV);
+#pragma unroll
+        for (int i = 0; i < 8; ++i) dst[i] = make_float4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 0) tmem_free(tmem, kTmemCols);
+}
+
+}  // namespace
+
+bool kda_chunk_tc_supports(int dk, int dv) { return dk == DK && dv == DV; }
+
+cudaError_t kda_launch_chunk_tc(const KdaChunkArgs &a, cudaStream_t stream) {
+    static bool configured[64] = {};
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    if (dev < 0 || dev >= 64 || !configured[dev]) {
+        e = cudaFuncSetAttribute(kda_chunk_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 (int)kSmemBytes);
+        if (e != cudaSuccess) return e;
+        if (dev >= 0 && dev < 64) configured[dev] = true;
+    }
+    const unsigned grid = (unsigned)((int64_t)a.N * a.H * NTILE);
+    kda_chunk_tc_kernel<<<grid, NTHR, kSmemBytes, stream>>>(a);
+    return cudaGetLastError();
+}
+
+cudaError_t kda_read_device_status(unsigned int *status, bool clear) {
+    cudaError_t e = cudaDeviceSynchronize();
+    if (e != cudaSuccess) return e;
+    e = cudaMemcpyFromSymbol(status, g_kda_device_status, sizeof(unsigned int));
+    if (e != cudaSuccess || !clear || *status == 0) return e;
+    const unsigned int zero = 0;
+    return cudaMemcpyToSymbol(g_kda_device_status, &zero, sizeof(unsigned int));
+}

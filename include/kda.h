@@ -113,6 +113,15 @@ int kda_decode_step(const void *q, const void *k, const void *v, const float *lo
                     const float *beta, float *S_inout, void *out, int N, int H, int dk,
                     int dv, int dtype, kda_stream_t stream);
 
+/*
+ * kda_device_status -- synchronises the current device, then reports whether any
+ * libkda kernel since the previous call gave up one of its bounded device-side
+ * waits (tensor-core completion barriers; each waits at most about two seconds
+ * and then abandons its work item instead of hanging).  Clears that record.
+ * Returns KDA_OK, KDA_ERR_TIMEOUT, or KDA_ERR_CUDA (the synchronisation failed).
+ */
+int kda_device_status(void);
+
 /* A static, human-readable description of a status code.  For KDA_ERR_CUDA it names
  * the CUDA error of the calling host thread's last failed launch. */
 const char *kda_status_string(int status);

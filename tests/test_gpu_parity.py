@@ -50,6 +50,8 @@ def check_against_oracle(inp, tol=None, tasks=None):
         ro = np.concatenate([x.ravel() for x in outs])
         eo = rel_err(go, ro)
         es = max(rel_err(S[n, h], s) for (n, h), s in zip(tasks, sts))
+    from gated_delta_rule_119_b200 import kda_device_status
+    assert kda_device_status() == 0, "a kernel gave up a bounded wait"
     assert eo <= tol, f"o: max rel err {eo:.3e} > {tol}"
     assert es <= tol, f"S_final: max rel err {es:.3e} > {tol}"
     return eo, es
