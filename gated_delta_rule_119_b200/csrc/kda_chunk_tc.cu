@@ -17,7 +17,8 @@
 // 64-127):  [u; o] = [T'; P T'] v + [-W; s q gamma - P W] S.
 //
 // Per chunk:
-//  E1  stage q, k (row-major) and the v slice (swizzled) in shared memory.
+//  E1  q, k (row-major) and the v slice (swizzled) arrive in shared memory by
+//      cp.async issued one chunk ahead; log_alpha is prefetched into registers.
 //  E2  one thread per (channel, pair of 16-row blocks): alpha = exp(log_alpha),
 //      block-local running products, and from them the operands k gamma,
 //      k kappa (tensor-core layout) and the factored operands of the 16 x 16
@@ -27,8 +28,8 @@
 //      [e^-70, e^70].  A diagonal block whose decay spread exceeds that range
 //      is handled per channel by exact running products instead.
 //  AP  A and P from those factors with warp-level bf16 MMAs (fp32 accumulation).
-//  T   T = (I + A)^{-1} by blocked forward substitution in fp32; T', P T'.
-//  TC  tcgen05: [W; P W] = [T'; P T'] (k gamma); state readout (bf16 copy,
+//  T   T = (I + A)^{-1} by blocked forward substitution in fp32.
+//  TC  tcgen05: [T'; P T'] = [I; P] T';  [W; P W] = [T'; P T'] (k gamma); state readout (bf16 copy,
 //      decay in place); [u; o] as above; S += (k kappa)^T u.
 #include <stdio.h>
 
@@ -51,13 +52,15 @@ constexpr long long kWaitCycles = 4000000000LL;   // about 2 s at B200 clocks
 constexpr uint32_t kTmemCols = 256;
 
 // Shared-memory map (bytes from a 1024-byte aligned base).
-constexpr uint32_t OFF_V = 0;                       // v slice, then u: 64 lines (MN-major B)
-constexpr uint32_t OFF_TP = OFF_V + 8192;           // [T'; P T']: 128 lines (K-major A)
+constexpr uint32_t OFF_V0 = 0;                      // v slice of even chunks, then their u (MN-major B)
+constexpr uint32_t OFF_V1 = OFF_V0 + 8192;          // the same for odd chunks
+constexpr uint32_t OFF_TP = OFF_V1 + 8192;          // [T'; P T']: 128 lines (K-major A)
 constexpr uint32_t OFF_KT = OFF_TP + 16384;         // k gamma: 2 x 64 lines (MN-major B)
 constexpr uint32_t OFF_KC = OFF_KT + 16384;         // k kappa: 2 x 64 lines (MN-major A)
-constexpr uint32_t OFF_X = OFF_KC + 16384;          // region X, reused:
+constexpr uint32_t OFF_X = OFF_KC + 16384;          // region X, reused within a chunk:
 constexpr uint32_t X_KL = 0, X_KR = 17408, X_TM = 34816, X_QL = 52224, X_SIZE = 69632;
-constexpr uint32_t X_A2 = 0, X_S = 32768;           //   later [-W; Q'] (2 x 128 lines) and S (128 lines)
+constexpr uint32_t X_IP = 0;                        //   [I; P] (128 lines) once KL is dead,
+constexpr uint32_t X_A2 = 0, X_S = 32768;           //   then [-W; Q'] (2 x 128 lines) and S (128 lines)
 constexpr uint32_t OFF_Q = OFF_X + X_SIZE;          // raw q [64][128] bf16
 constexpr uint32_t OFF_K = OFF_Q + 16384;           // raw k
 constexpr uint32_t OFF_AM = OFF_K + 16384;          // A [64][LF] fp32
@@ -80,20 +83,74 @@ __constant__ int kPairA[10] = {0, 1, 1, 2, 2, 2, 3, 3, 3, 3};
 __constant__ int kPairB[10] = {0, 0, 1, 0, 1, 2, 0, 1, 2, 3};
 
 __device__ __forceinline__ float bf(const __nv_bfloat16 *p) { return __bfloat162float(*p); }
+__device__ __forceinline__ float2 bf2(const __nv_bfloat16 *p) {
+    return __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(p));
+}
+__device__ __forceinline__ void st_bf2(void *p, float x, float y) {
+    *reinterpret_cast<uint32_t *>(p) = pack_bf16(x, y);
+}
+
+struct ChunkPos {
+    int64_t c0;
+    int nr;
+};
+
+__device__ __forceinline__ ChunkPos chunk_pos(int64_t t0, int64_t t1, int ci) {
+    const int64_t c0 = t0 + (int64_t)ci * CH;
+    return {c0, (int)(t1 - c0 < CH ? t1 - c0 : CH)};
+}
+
+// Stage q and k rows [c0, c0 + 64) (rows past the sequence end read as zero).
+__device__ __forceinline__ void issue_qk(uint8_t *sm, const __nv_bfloat16 *qg, const __nv_bfloat16 *kg,
+                                         ChunkPos cp, int H, int h, int tid) {
+    for (int idx = tid; idx < 2048; idx += NTHR) {
+        const int which = idx >> 10, rem = idx & 1023, r = rem >> 4, j = rem & 15;
+        const int rs = r < cp.nr ? r : cp.nr - 1;
+        const __nv_bfloat16 *src = (which ? kg : qg) + ((size_t)(cp.c0 + rs) * H + h) * DK + j * 8;
+        cp_async16(sm + (which ? OFF_K : OFF_Q) + r * 256 + j * 16, src, r < cp.nr ? 16u : 0u);
+    }
+}
+__device__ __forceinline__ void issue_v(uint8_t *dst, const __nv_bfloat16 *vg, ChunkPos cp, int H,
+                                        int h, int tile, int tid) {
+    for (int idx = tid; idx < 512; idx += NTHR) {
+        const int r = idx >> 3, j = idx & 7;
+        const int rs = r < cp.nr ? r : cp.nr - 1;
+        const __nv_bfloat16 *src = vg + ((size_t)(cp.c0 + rs) * H + h) * DV + tile * DVT + j * 8;
+        cp_async16(dst + sw128_chunk(r, j), src, r < cp.nr ? 16u : 0u);
+    }
+}
+// log_alpha of 16 rows x 2 channels for E2 (zero past the sequence end).
+__device__ __forceinline__ void load_la(float2 *la, const float *lag, ChunkPos cp, int H, int h, int b,
+                                        int c2) {
+#pragma unroll
+    for (int rr = 0; rr < 16; ++rr) {
+        const int r = 16 * b + rr;
+        la[rr] = r < cp.nr ? *reinterpret_cast<const float2 *>(lag + ((size_t)(cp.c0 + r) * H + h) * DK + c2)
+                           : make_float2(0.f, 0.f);
+    }
+}
+__device__ __forceinline__ uint4 pack8(const float *v) {
+    uint4 pk;
+    pk.x = pack_bf16(v[0], v[1]);
+    pk.y = pack_bf16(v[2], v[3]);
+    pk.z = pack_bf16(v[4], v[5]);
+    pk.w = pack_bf16(v[6], v[7]);
+    return pk;
+}
 
 __global__ void __launch_bounds__(NTHR, 1) kda_chunk_tc_kernel(KdaChunkArgs a) {
     extern __shared__ uint8_t smraw[];
     uint8_t *sm = (uint8_t *)(((uintptr_t)smraw + 1023) & ~(uintptr_t)1023);
-    __shared__ uint64_t bar_w, bar_uo, bar_s;
+    __shared__ uint64_t bar_p, bar_w, bar_uo, bar_s;
     __shared__ uint32_t s_tmem;
     __shared__ int s_abort;
 
-    uint8_t *sV = sm + OFF_V, *sTP = sm + OFF_TP, *sKt = sm + OFF_KT, *sKC = sm + OFF_KC;
+    uint8_t *sTP = sm + OFF_TP, *sKt = sm + OFF_KT, *sKC = sm + OFF_KC;
     uint8_t *sX = sm + OFF_X;
     __nv_bfloat16 *KL = (__nv_bfloat16 *)(sX + X_KL), *KR = (__nv_bfloat16 *)(sX + X_KR);
     __nv_bfloat16 *QL = (__nv_bfloat16 *)(sX + X_QL);
     float *Tm = (float *)(sX + X_TM);
-    uint8_t *sA2 = sX + X_A2, *sS = sX + X_S;
+    uint8_t *sIP = sX + X_IP, *sA2 = sX + X_A2, *sS = sX + X_S;
     const __nv_bfloat16 *sQ = (const __nv_bfloat16 *)(sm + OFF_Q);
     const __nv_bfloat16 *sK = (const __nv_bfloat16 *)(sm + OFF_K);
     float *Am = (float *)(sm + OFF_AM), *Pm = (float *)(sm + OFF_PM);
@@ -112,8 +169,22 @@ __global__ void __launch_bounds__(NTHR, 1) kda_chunk_tc_kernel(KdaChunkArgs a) {
     __nv_bfloat16 *og = static_cast<__nv_bfloat16 *>(a.out);
     int64_t t0, t1;
     kda::seq_bounds(a.cu_seqlens, n, a.T, a.T_total, t0, t1);
+    const int nchunks = (int)((t1 - t0 + CH - 1) / CH);
+
+    // E2 thread mapping: channels {2 c2h, 2 c2h + 1} of 16-row block eb.
+    const int c2 = 2 * (tid & 63), eb = tid >> 6;
+    float2 la[16];
+    if (nchunks > 0) {
+        const ChunkPos cp0 = chunk_pos(t0, t1, 0);
+        issue_qk(sm, qg, kg, cp0, H, h, tid);
+        asm volatile("cp.async.commit_group;" ::: "memory");
+        issue_v(sm + OFF_V0, vg, cp0, H, h, tile, tid);
+        asm volatile("cp.async.commit_group;" ::: "memory");
+        load_la(la, a.log_alpha, cp0, H, h, eb, c2);
+    }
 
     if (tid == 0) {
+        mbar_init(&bar_p, 1);
         mbar_init(&bar_w, 1);
         mbar_init(&bar_uo, 1);
         mbar_init(&bar_s, 1);
@@ -150,126 +221,135 @@ __global__ void __launch_bounds__(NTHR, 1) kda_chunk_tc_kernel(KdaChunkArgs a) {
     __syncthreads();
     tc_fence_after();
 
-    const int nchunks = (int)((t1 - t0 + CH - 1) / CH);
     uint64_t *pending = nullptr;
     uint32_t pending_par = 0;
     for (int ci = 0; ci < nchunks; ++ci) {
         const uint32_t par = (uint32_t)(ci & 1);
-        const int64_t c0 = t0 + (int64_t)ci * CH;
-        const int nr = (int)(t1 - c0 < CH ? t1 - c0 : CH);
+        const ChunkPos cp = chunk_pos(t0, t1, ci);
+        const int64_t c0 = cp.c0;
+        const int nr = cp.nr;
+        uint8_t *sV = sm + (par ? OFF_V1 : OFF_V0);
 
-        // ---------------- E1: stage q, k, v slice, beta; clear the diagonal blocks of A, P
-        for (int idx = tid; idx < 2048; idx += NTHR) {
-            const int which = idx >> 10, rem = idx & 1023, r = rem >> 4, j = rem & 15;
-            const int rs = r < nr ? r : nr - 1;
-            const __nv_bfloat16 *src = (which ? kg : qg) + ((size_t)(c0 + rs) * H + h) * DK + j * 8;
-            cp_async16(sm + (which ? OFF_K : OFF_Q) + r * 256 + j * 16, src, r < nr ? 16u : 0u);
-        }
-        for (int idx = tid; idx < 512; idx += NTHR) {
-            const int r = idx >> 3, j = idx & 7;
-            const int rs = r < nr ? r : nr - 1;
-            const __nv_bfloat16 *src = vg + ((size_t)(c0 + rs) * H + h) * DV + tile * DVT + j * 8;
-            cp_async16(sV + sw128_chunk(r, j), src, r < nr ? 16u : 0u);
-        }
+        // ---------------- E1: prefetch the next v slice; wait for this chunk's q, k, v
+        if (ci + 1 < nchunks)
+            issue_v(sm + (par ? OFF_V0 : OFF_V1), vg, chunk_pos(t0, t1, ci + 1), H, h, tile, tid);
+        asm volatile("cp.async.commit_group;" ::: "memory");
         if (tid < CH) sBeta[tid] = tid < nr ? a.beta[(size_t)(c0 + tid) * H + h] : 0.f;
         for (int idx = tid; idx < 2048; idx += NTHR) {
             const int m = idx >> 10, rem = idx & 1023, blk = rem >> 8, r = (rem >> 4) & 15, i = rem & 15;
             (m ? Pm : Am)[(16 * blk + r) * LF + 16 * blk + i] = 0.f;
         }
-        cp_async_wait_all();
+        asm volatile("cp.async.wait_group 1;" ::: "memory");
         __syncthreads();
 
         // ---------------- E2 pass 1: alpha, per-block sums and products
-        const int ch = tid & 127, hb = tid >> 7;     // channel, pair of blocks {2hb, 2hb+1}
-        float al[32];
-#pragma unroll
-        for (int rr = 0; rr < 32; ++rr) {
-            const int r = 32 * hb + rr;
-            al[rr] = r < nr ? a.log_alpha[((size_t)(c0 + r) * H + h) * DK + ch] : 0.f;
-        }
-#pragma unroll
-        for (int bb = 0; bb < 2; ++bb) {
-            float s = 0.f, p = 1.f;
+        {
+            float s0 = 0.f, s1 = 0.f, p0 = 1.f, p1 = 1.f;
 #pragma unroll
             for (int rr = 0; rr < 16; ++rr) {
-                const float la = al[16 * bb + rr];
-                s += la;
-                const float x = expf(la);
-                al[16 * bb + rr] = x;
-                p *= x;
+                s0 += la[rr].x;
+                s1 += la[rr].y;
+                la[rr].x = expf(la[rr].x);
+                la[rr].y = expf(la[rr].y);
+                p0 *= la[rr].x;
+                p1 *= la[rr].y;
             }
-            sBS[(2 * hb + bb) * 128 + ch] = s;
-            sBT[(2 * hb + bb) * 128 + ch] = p;
+            *reinterpret_cast<float2 *>(&sBS[eb * 128 + c2]) = make_float2(s0, s1);
+            *reinterpret_cast<float2 *>(&sBT[eb * 128 + c2]) = make_float2(p0, p1);
         }
         __syncthreads();
 
-        // ---------------- E2 pass 2: operands
-#pragma unroll
-        for (int bb = 0; bb < 2; ++bb) {
-            const int b = 2 * hb + bb;
-            float gpre = 1.f, ksuf = 1.f;
+        // ---------------- E2 pass 2: operands (alpha now in la)
+        {
+            float2 gpre = make_float2(1.f, 1.f), ksuf = make_float2(1.f, 1.f);
 #pragma unroll
             for (int j = 0; j < 4; ++j) {
-                if (j < b) gpre *= sBT[j * 128 + ch];
-                if (j > b) ksuf *= sBT[j * 128 + ch];
+                const float2 bt = *reinterpret_cast<const float2 *>(&sBT[j * 128 + c2]);
+                if (j < eb) { gpre.x *= bt.x; gpre.y *= bt.y; }
+                if (j > eb) { ksuf.x *= bt.x; ksuf.y *= bt.y; }
             }
-            const float bs = sBS[b * 128 + ch];
-            const bool flagged = bs < -kSpreadLimit;
-            const float rho = flagged ? 1.f : expf(-0.5f * bs);
-            sQF[b * 128 + ch] = flagged ? gpre : gpre * expf(0.5f * bs);
-            const uint32_t blk_off = (uint32_t)(ch >> 6) * 8192u;
-            float lam = 1.f;
+            const float2 bs = *reinterpret_cast<const float2 *>(&sBS[eb * 128 + c2]);
+            const bool fl0 = bs.x < -kSpreadLimit, fl1 = bs.y < -kSpreadLimit;
+            const float rho0 = fl0 ? 1.f : expf(-0.5f * bs.x), rho1 = fl1 ? 1.f : expf(-0.5f * bs.y);
+            *reinterpret_cast<float2 *>(&sQF[eb * 128 + c2]) =
+                make_float2(fl0 ? gpre.x : gpre.x * expf(0.5f * bs.x), fl1 ? gpre.y : gpre.y * expf(0.5f * bs.y));
+            const uint32_t col_off = (uint32_t)(c2 >> 6) * 8192u;
+            float l0 = 1.f, l1 = 1.f;
 #pragma unroll
             for (int rr = 0; rr < 16; ++rr) {
-                const int r = 16 * b + rr;
-                lam *= al[16 * bb + rr];
-                const float kv = bf(&sK[r * 128 + ch]), qv = bf(&sQ[r * 128 + ch]);
-                *(__nv_bfloat16 *)(sKt + blk_off + sw128(r, ch & 63)) = __float2bfloat16_rn(kv * (gpre * lam));
-                KL[r * LP + ch] = __float2bfloat16_rn(kv * (rho * lam));
-                QL[r * LP + ch] = __float2bfloat16_rn(scale * qv * (rho * lam));
+                const int r = 16 * eb + rr;
+                l0 *= la[rr].x;
+                l1 *= la[rr].y;
+                const float2 kv = bf2(&sK[r * 128 + c2]), qv = bf2(&sQ[r * 128 + c2]);
+                st_bf2(sKt + col_off + sw128(r, c2 & 63), kv.x * (gpre.x * l0), kv.y * (gpre.y * l1));
+                st_bf2(&KL[r * LP + c2], kv.x * (rho0 * l0), kv.y * (rho1 * l1));
+                st_bf2(&QL[r * LP + c2], scale * qv.x * (rho0 * l0), scale * qv.y * (rho1 * l1));
             }
-            float sig = 1.f;
+            float g0 = 1.f, g1 = 1.f;
 #pragma unroll
             for (int rr = 15; rr >= 0; --rr) {
-                const int r = 16 * b + rr;
-                const float kv = bf(&sK[r * 128 + ch]);
-                *(__nv_bfloat16 *)(sKC + blk_off + sw128(r, ch & 63)) = __float2bfloat16_rn(kv * (sig * ksuf));
-                KR[r * LP + ch] = __float2bfloat16_rn(kv * (rho * sig));
-                sig *= al[16 * bb + rr];
+                const int r = 16 * eb + rr;
+                const float2 kv = bf2(&sK[r * 128 + c2]);
+                st_bf2(sKC + col_off + sw128(r, c2 & 63), kv.x * (g0 * ksuf.x), kv.y * (g1 * ksuf.y));
+                st_bf2(&KR[r * LP + c2], kv.x * (rho0 * g0), kv.y * (rho1 * g1));
+                g0 *= la[rr].x;
+                g1 *= la[rr].y;
             }
-            if (flagged) {
-                // Exact diagonal-block contribution of this channel (running products).
+            if (fl0 || fl1) {
+                // Exact diagonal-block contribution of a flagged channel (running products).
 #pragma unroll
-                for (int i = 0; i < 16; ++i) {
-                    const float ki = bf(&sK[(16 * b + i) * 128 + ch]);
-                    float f = 1.f;
+                for (int cc = 0; cc < 2; ++cc) {
+                    if (!(cc ? fl1 : fl0)) continue;
+                    const int ch = c2 + cc;
 #pragma unroll
-                    for (int r = i; r < 16; ++r) {
-                        if (r > i) f *= al[16 * bb + r];
-                        const int R = 16 * b + r, I = 16 * b + i;
-                        const float kd = ki * f;
-                        if (r > i) atomicAdd(&Am[R * LF + I], sBeta[R] * bf(&sK[R * 128 + ch]) * kd);
-                        atomicAdd(&Pm[R * LF + I], scale * bf(&sQ[R * 128 + ch]) * kd);
+                    for (int i = 0; i < 16; ++i) {
+                        const float ki = bf(&sK[(16 * eb + i) * 128 + ch]);
+                        float f = 1.f;
+#pragma unroll
+                        for (int r = i; r < 16; ++r) {
+                            if (r > i) f *= cc ? la[r].y : la[r].x;
+                            const int R = 16 * eb + r, I = 16 * eb + i;
+                            const float kd = ki * f;
+                            if (r > i) atomicAdd(&Am[R * LF + I], sBeta[R] * bf(&sK[R * 128 + ch]) * kd);
+                            atomicAdd(&Pm[R * LF + I], scale * bf(&sQ[R * 128 + ch]) * kd);
+                        }
                     }
                 }
             }
-        }
-        if (hb == 0) sGC[ch] = sBT[ch] * sBT[128 + ch] * sBT[256 + ch] * sBT[384 + ch];
+            if (eb == 0) {
+                float2 gc = make_float2(1.f, 1.f);
 #pragma unroll
-        for (int pp = 0; pp < 5; ++pp) {
-            const int p = 5 * hb + pp, pa = kPairA[p], pb = kPairB[p];
-            float sc;
-            const bool fa = sBS[pa * 128 + ch] < -kSpreadLimit, fb = sBS[pb * 128 + ch] < -kSpreadLimit;
-            if (pa == pb) {
-                sc = fa ? 0.f : 1.f;
-            } else {
-                float e = (fa ? 0.f : 0.5f * sBS[pa * 128 + ch]) + (fb ? 0.f : 0.5f * sBS[pb * 128 + ch]);
-                for (int j = pb + 1; j < pa; ++j) e += sBS[j * 128 + ch];
-                sc = expf(e);
+                for (int j = 0; j < 4; ++j) {
+                    const float2 bt = *reinterpret_cast<const float2 *>(&sBT[j * 128 + c2]);
+                    gc.x *= bt.x;
+                    gc.y *= bt.y;
+                }
+                *reinterpret_cast<float2 *>(&sGC[c2]) = gc;
             }
-            sSC[p * 128 + ch] = sc;
+#pragma unroll
+            for (int k5 = 0; k5 < 5; ++k5) {
+                const int e = tid + NTHR * k5, p = e >> 7, ch = e & 127, pa = kPairA[p], pb = kPairB[p];
+                const float bsa = sBS[pa * 128 + ch], bsb = sBS[pb * 128 + ch];
+                const bool fa = bsa < -kSpreadLimit, fb = bsb < -kSpreadLimit;
+                float sc;
+                if (pa == pb) {
+                    sc = fa ? 0.f : 1.f;
+                } else {
+                    float ex = (fa ? 0.f : 0.5f * bsa) + (fb ? 0.f : 0.5f * bsb);
+                    for (int j = pb + 1; j < pa; ++j) ex += sBS[j * 128 + ch];
+                    sc = expf(ex);
+                }
+                sSC[p * 128 + ch] = sc;
+            }
         }
         __syncthreads();
+        // q, k of the next chunk can now replace this chunk's; log_alpha into registers.
+        if (ci + 1 < nchunks) {
+            const ChunkPos cn = chunk_pos(t0, t1, ci + 1);
+            issue_qk(sm, qg, kg, cn, H, h, tid);
+            load_la(la, a.log_alpha, cn, H, h, eb, c2);
+        }
+        asm volatile("cp.async.commit_group;" ::: "memory");
 
         // ---------------- AP: 16 x 16 blocks of A and P with warp MMAs
         {
@@ -277,7 +357,7 @@ __global__ void __launch_bounds__(NTHR, 1) kda_chunk_tc_kernel(KdaChunkArgs a) {
             for (int task = warp; task < 20; task += 8) {
                 const int mat = task / 10, p = task % 10, pa = kPairA[p], pb = kPairB[p];
                 const __nv_bfloat16 *Ls = mat == 0 ? KL : QL;
-                float acc[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+                float acc[2][2][4] = {};
 #pragma unroll
                 for (int kt = 0; kt < 8; ++kt) {
                     const int c = 16 * kt + 2 * t4;
@@ -285,15 +365,15 @@ __global__ void __launch_bounds__(NTHR, 1) kda_chunk_tc_kernel(KdaChunkArgs a) {
                     const uint32_t a1 = *(const uint32_t *)&Ls[(16 * pa + g + 8) * LP + c];
                     const uint32_t a2 = *(const uint32_t *)&Ls[(16 * pa + g) * LP + c + 8];
                     const uint32_t a3 = *(const uint32_t *)&Ls[(16 * pa + g + 8) * LP + c + 8];
-                    const float s0 = sSC[p * 128 + c], s1 = sSC[p * 128 + c + 1];
-                    const float s8 = sSC[p * 128 + c + 8], s9 = sSC[p * 128 + c + 9];
+                    const float2 s01 = *reinterpret_cast<const float2 *>(&sSC[p * 128 + c]);
+                    const float2 s89 = *reinterpret_cast<const float2 *>(&sSC[p * 128 + c + 8]);
 #pragma unroll
                     for (int j = 0; j < 2; ++j) {
                         const int i = 16 * pb + 8 * j + g;
                         const float2 f0 = unpack_bf16(*(const uint32_t *)&KR[i * LP + c]);
                         const float2 f1 = unpack_bf16(*(const uint32_t *)&KR[i * LP + c + 8]);
-                        mma_m16n8k16(acc[j], a0, a1, a2, a3, pack_bf16(f0.x * s0, f0.y * s1),
-                                     pack_bf16(f1.x * s8, f1.y * s9));
+                        mma_m16n8k16(acc[kt & 1][j], a0, a1, a2, a3, pack_bf16(f0.x * s01.x, f0.y * s01.y),
+                                     pack_bf16(f1.x * s89.x, f1.y * s89.y));
                     }
                 }
 #pragma unroll
@@ -302,7 +382,7 @@ __global__ void __launch_bounds__(NTHR, 1) kda_chunk_tc_kernel(KdaChunkArgs a) {
                     for (int e = 0; e < 4; ++e) {
                         const int r = 16 * pa + g + (e >= 2 ? 8 : 0);
                         const int i = 16 * pb + 8 * j + 2 * t4 + (e & 1);
-                        const float val = acc[j][e];
+                        const float val = acc[0][j][e] + acc[1][j][e];
                         if (mat == 0) {
                             if (pa != pb) Am[r * LF + i] = sBeta[r] * val;
                             else if (i < r) Am[r * LF + i] += sBeta[r] * val;
@@ -325,11 +405,15 @@ __global__ void __launch_bounds__(NTHR, 1) kda_chunk_tc_kernel(KdaChunkArgs a) {
             for (int r = 0; r < 16; ++r) {
                 float s = r == i ? 1.f : 0.f;
                 if (r > i) {
-                    float acc = 0.f;
+                    float acc0 = 0.f, acc1 = 0.f;
 #pragma unroll
-                    for (int m = 0; m < r; ++m)
-                        if (m >= i) acc = fmaf(Ab[r * LF + m], tc[m], acc);
-                    s = -acc;
+                    for (int m = 0; m < r; ++m) {
+                        if (m >= i) {
+                            if (m & 1) acc1 = fmaf(Ab[r * LF + m], tc[m], acc1);
+                            else acc0 = fmaf(Ab[r * LF + m], tc[m], acc0);
+                        }
+                    }
+                    s = -(acc0 + acc1);
                 }
                 tc[r] = s;
             }
@@ -338,42 +422,99 @@ __global__ void __launch_bounds__(NTHR, 1) kda_chunk_tc_kernel(KdaChunkArgs a) {
         }
         __syncthreads();
         //      off-diagonal blocks, by distance d = a - b: T_ab = -T_aa sum_{m=b}^{a-1} A_am T_mb
-        for (int d = 1; d < 4; ++d) {
-            const int nblk = 4 - d;
-            for (int o = tid; o < nblk * 256; o += NTHR) {
-                const int b = o >> 8, pa = b + d, rr = (o >> 4) & 15, ii = o & 15;
-                float x = 0.f;
-                for (int m = b; m < pa; ++m) {
-                    const float *arow = Am + (16 * pa + rr) * LF + 16 * m;
-                    const float *tcol = Tm + (16 * m) * LF + 16 * b + ii;
+        {
+            const int rr = tid >> 4, ii = tid & 15;
+            for (int d = 1; d < 4; ++d) {
+                const int nblk = 4 - d;
 #pragma unroll
-                    for (int jj = 0; jj < 16; ++jj) x = fmaf(arow[jj], tcol[jj * LF], x);
+                for (int b = 0; b < 3; ++b) {
+                    if (b < nblk) {
+                        const int pa = b + d;
+                        float x[4] = {0.f, 0.f, 0.f, 0.f};
+                        for (int m = b; m < pa; ++m) {
+                            const float *arow = Am + (16 * pa + rr) * LF + 16 * m;
+                            const float *tcol = Tm + (16 * m) * LF + 16 * b + ii;
+#pragma unroll
+                            for (int jj = 0; jj < 16; ++jj) x[jj & 3] = fmaf(arow[jj], tcol[jj * LF], x[jj & 3]);
+                        }
+                        sXT[(b << 8) + tid] = (x[0] + x[1]) + (x[2] + x[3]);
+                    }
                 }
-                sXT[o] = x;
+                __syncthreads();
+#pragma unroll
+                for (int b = 0; b < 3; ++b) {
+                    if (b < nblk) {
+                        const int pa = b + d;
+                        const float *trow_ = Tm + (16 * pa + rr) * LF + 16 * pa;
+                        const float *xcol = sXT + (b << 8) + ii;
+                        float x[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+                        for (int jj = 0; jj < 16; ++jj)
+                            if (jj <= rr) x[jj & 3] = fmaf(trow_[jj], xcol[jj * 16], x[jj & 3]);
+                        Tm[(16 * pa + rr) * LF + 16 * b + ii] = -((x[0] + x[1]) + (x[2] + x[3]));
+                    }
+                }
+                __syncthreads();
             }
-            __syncthreads();
-            for (int o = tid; o < nblk * 256; o += NTHR) {
-                const int b = o >> 8, pa = b + d, rr = (o >> 4) & 15, ii = o & 15;
-                const float *trow_ = Tm + (16 * pa + rr) * LF + 16 * pa;
-                const float *xcol = sXT + (b << 8) + ii;
-                float x = 0.f;
-                for (int jj = 0; jj <= rr; ++jj) x = fmaf(trow_[jj], xcol[jj * 16], x);
-                Tm[(16 * pa + rr) * LF + 16 * b + ii] = -x;
-            }
-            __syncthreads();
         }
-        //      [T'; P T'] -> tensor-core operand (K-major, 128 lines)
-        for (int o = tid; o < CH * CH; o += NTHR) {
-            const int r = o >> 6, i = o & 63;
-            const float tv = i <= r ? Tm[r * LF + i] * sBeta[i] : 0.f;
-            *(__nv_bfloat16 *)(sTP + sw128(r, i)) = __float2bfloat16_rn(tv);
-            float pv = 0.f;
-            for (int m = i; m <= r; ++m) pv = fmaf(Pm[r * LF + m], Tm[m * LF + i], pv);
-            *(__nv_bfloat16 *)(sTP + sw128(64 + r, i)) = __float2bfloat16_rn(i <= r ? pv * sBeta[i] : 0.f);
+        //      T' (lines 0-63 of [T'; P T']) and [I; P] as tensor-core operands, 8 elements at a time
+        for (int o = tid; o < 1536; o += NTHR) {
+            const int l = o >> 3, j = o & 7;     // l < 64: T' line; else [I; P] line l - 64
+            float v8[8];
+            if (l < 64) {
+#pragma unroll
+                for (int e = 0; e < 8; ++e) {
+                    const int i = 8 * j + e;
+                    v8[e] = i <= l ? Tm[l * LF + i] * sBeta[i] : 0.f;
+                }
+                *(uint4 *)(sTP + sw128_chunk(l, j)) = pack8(v8);
+            } else {
+                const int pl = l - 64;          // line of [I; P]
+#pragma unroll
+                for (int e = 0; e < 8; ++e) {
+                    const int i = 8 * j + e;
+                    v8[e] = pl < 64 ? (i == pl ? 1.f : 0.f) : (i <= pl - 64 ? Pm[(pl - 64) * LF + i] : 0.f);
+                }
+                *(uint4 *)(sIP + sw128_chunk(pl, j)) = pack8(v8);
+            }
         }
         fence_async_smem();
         tc_fence_before();
         __syncthreads();
+        tc_fence_after();
+
+        // ---------------- TC: [T'; P T'] = [I; P] T'   (into the [u; o] columns, free here)
+        if (tid == 0) {
+            const uint32_t ip = smem_u32(sIP), tp = smem_u32(sTP);
+#pragma unroll
+            for (int ks = 0; ks < 4; ++ks)
+                mma_bf16(T_UO, desc_sw128(ip + 32 * ks, 16, 1024), desc_sw128(tp + 2048 * ks, 8192, 1024),
+                         idesc_bf16(128, 64, false, true), ks > 0);
+            mma_commit(&bar_p);
+        }
+        //      state slice: bf16 copy for the MMAs, decay in place for the update
+        {
+            float v[32];
+            tmem_ld32(T_S + lane_off + half * 32, v);
+#pragma unroll
+            for (int m = 0; m < 4; ++m) *(uint4 *)(sS + sw128_chunk(trow, 4 * half + m)) = pack8(v + 8 * m);
+            const float gdec = sGC[trow];
+#pragma unroll
+            for (int i = 0; i < 32; ++i) v[i] *= gdec;
+            tmem_st32(T_S + lane_off + half * 32, v);
+        }
+        if (!mbar_wait(&bar_p, par, kWaitCycles)) s_abort = 1;
+        tc_fence_after();
+        if (trow >= 64) {
+            float v[32];
+            tmem_ld32(T_UO + lane_off + half * 32, v);
+#pragma unroll
+            for (int m = 0; m < 4; ++m) *(uint4 *)(sTP + sw128_chunk(trow, 4 * half + m)) = pack8(v + 8 * m);
+        }
+        fence_async_smem();
+        tc_fence_before();
+        __syncthreads();
+        if (s_abort) { pending = &bar_p; pending_par = par; break; }
         tc_fence_after();
 
         // ---------------- TC: [W; P W] = [T'; P T'] (k gamma)
@@ -384,24 +525,6 @@ __global__ void __launch_bounds__(NTHR, 1) kda_chunk_tc_kernel(KdaChunkArgs a) {
                 mma_bf16(T_W, desc_sw128(a0 + 32 * ks, 16, 1024), desc_sw128(b0 + 2048 * ks, 8192, 1024),
                          idesc_bf16(128, 128, false, true), ks > 0);
             mma_commit(&bar_w);
-        }
-        //      state slice: bf16 copy for the MMAs, decay in place for the update
-        {
-            float v[32];
-            tmem_ld32(T_S + lane_off + half * 32, v);
-#pragma unroll
-            for (int m = 0; m < 4; ++m) {
-                uint4 pk;
-                pk.x = pack_bf16(v[8 * m + 0], v[8 * m + 1]);
-                pk.y = pack_bf16(v[8 * m + 2], v[8 * m + 3]);
-                pk.z = pack_bf16(v[8 * m + 4], v[8 * m + 5]);
-                pk.w = pack_bf16(v[8 * m + 6], v[8 * m + 7]);
-                *(uint4 *)(sS + sw128_chunk(trow, 4 * half + m)) = pk;
-            }
-            const float gdec = sGC[trow];
-#pragma unroll
-            for (int i = 0; i < 32; ++i) v[i] *= gdec;
-            tmem_st32(T_S + lane_off + half * 32, v);
         }
         if (!mbar_wait(&bar_w, par, kWaitCycles)) s_abort = 1;
         tc_fence_after();
@@ -416,20 +539,18 @@ __global__ void __launch_bounds__(NTHR, 1) kda_chunk_tc_kernel(KdaChunkArgs a) {
                     const int r = trow - 64;
                     const float *qf = sQF + (r >> 4) * 128 + c0c;
 #pragma unroll
-                    for (int i = 0; i < 32; ++i) v[i] = bf(&QL[r * LP + c0c + i]) * qf[i] - v[i];
+                    for (int i = 0; i < 32; i += 2) {
+                        const float2 ql = bf2(&QL[r * LP + c0c + i]);
+                        v[i] = ql.x * qf[i] - v[i];
+                        v[i + 1] = ql.y * qf[i + 1] - v[i + 1];
+                    }
                 } else {
 #pragma unroll
                     for (int i = 0; i < 32; ++i) v[i] = -v[i];
                 }
 #pragma unroll
-                for (int m = 0; m < 4; ++m) {
-                    uint4 pk;
-                    pk.x = pack_bf16(v[8 * m + 0], v[8 * m + 1]);
-                    pk.y = pack_bf16(v[8 * m + 2], v[8 * m + 3]);
-                    pk.z = pack_bf16(v[8 * m + 4], v[8 * m + 5]);
-                    pk.w = pack_bf16(v[8 * m + 6], v[8 * m + 7]);
-                    *(uint4 *)(sA2 + half * 16384 + sw128_chunk(trow, 4 * part + m)) = pk;
-                }
+                for (int m = 0; m < 4; ++m)
+                    *(uint4 *)(sA2 + half * 16384 + sw128_chunk(trow, 4 * part + m)) = pack8(v + 8 * m);
             }
         }
         fence_async_smem();
@@ -459,12 +580,7 @@ __global__ void __launch_bounds__(NTHR, 1) kda_chunk_tc_kernel(KdaChunkArgs a) {
             tmem_ld32(T_UO + lane_off + half * 32, v);
             uint4 pk[4];
 #pragma unroll
-            for (int m = 0; m < 4; ++m) {
-                pk[m].x = pack_bf16(v[8 * m + 0], v[8 * m + 1]);
-                pk[m].y = pack_bf16(v[8 * m + 2], v[8 * m + 3]);
-                pk[m].z = pack_bf16(v[8 * m + 4], v[8 * m + 5]);
-                pk[m].w = pack_bf16(v[8 * m + 6], v[8 * m + 7]);
-            }
+            for (int m = 0; m < 4; ++m) pk[m] = pack8(v + 8 * m);
             if (trow < 64) {
 #pragma unroll
                 for (int m = 0; m < 4; ++m) *(uint4 *)(sV + sw128_chunk(trow, 4 * half + m)) = pk[m];
@@ -495,6 +611,7 @@ __global__ void __launch_bounds__(NTHR, 1) kda_chunk_tc_kernel(KdaChunkArgs a) {
         __syncthreads();
         if (s_abort) { pending = &bar_s; pending_par = par; break; }
     }
+    asm volatile("cp.async.wait_all;" ::: "memory");
 
     if (pending) {
         // A tensor-core wait gave up: record it, give the in-flight work one more

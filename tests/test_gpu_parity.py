@@ -52,6 +52,8 @@ def check_against_oracle(inp, tol=None, tasks=None):
         es = max(rel_err(S[n, h], s) for (n, h), s in zip(tasks, sts))
     from gated_delta_rule_119_b200 import kda_device_status
     assert kda_device_status() == 0, "a kernel gave up a bounded wait"
+    print(f"[parity] {inp.dtype} T={inp.total_tokens} H={inp.H} dk={inp.dk} dv={inp.dv} "
+          f"gates={inp.meta.get('gates')}: o {eo:.3e}  S_final {es:.3e}")
     assert eo <= tol, f"o: max rel err {eo:.3e} > {tol}"
     assert es <= tol, f"S_final: max rel err {es:.3e} > {tol}"
     return eo, es
