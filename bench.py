@@ -162,7 +162,8 @@ def source_digest(rel: str) -> str:
 def profiled_traffic(kernel_key: str, workload: str):
     """DRAM bytes per launch recorded in a committed ncu summary, or None when
     there is none or the kernel source changed since it was taken."""
-    path = os.path.join(PROFILES, f"traffic_{kernel_key}_{workload}.md")
+    stem = os.path.splitext(os.path.basename(KERNEL_SOURCES[kernel_key]))[0]
+    path = os.path.join(PROFILES, f"{stem}__{workload}.md")
     if not os.path.exists(path):
         return None
     text = open(path).read()
