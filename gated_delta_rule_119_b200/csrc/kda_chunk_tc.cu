@@ -257,8 +257,8 @@ __global__ void __launch_bounds__(NTHR, 1) kda_chunk_tc_kernel(KdaChunkArgs a) {
             for (int rr = 0; rr < 16; ++rr) {
                 s0 += la[rr].x;
                 s1 += la[rr].y;
-                la[rr].x = expf(la[rr].x);
-                la[rr].y = expf(la[rr].y);
+                la[rr].x = __expf(la[rr].x);
+                la[rr].y = __expf(la[rr].y);
                 p0 *= la[rr].x;
                 p1 *= la[rr].y;
             }
@@ -286,13 +286,14 @@ __global__ void __launch_bounds__(NTHR, 1) kda_chunk_tc_kernel(KdaChunkArgs a) {
                 if (j > eb) { ksuf.x *= bt.x; ksuf.y *= bt.y; }
             }
             if (fast) {   // k e^-g = k kappa e^{-g_last}
-                ksuf.x *= expf(-gsum.x);
-                ksuf.y *= expf(-gsum.y);
+                ksuf.x *= __expf(-gsum.x);
+                ksuf.y *= __expf(-gsum.y);
             }
             const uint32_t col_kq = (uint32_t)(c2 >> 6) * 16384u, col_kc = (uint32_t)(c2 >> 6) * 8192u;
             const float2 bs = *reinterpret_cast<const float2 *>(&sBS[eb * 128 + c2]);
             const bool fl0 = bs.x < -kSpreadLimit, fl1 = bs.y < -kSpreadLimit;
-            const float rho0 = fl0 ? 1.f : expf(-0.5f * bs.x), rho1 = fl1 ? 1.f : expf(-0.5f * bs.y);
+            const float rho0 = fast || fl0 ? 1.f : __expf(-0.5f * bs.x);
+            const float rho1 = fast || fl1 ? 1.f : __expf(-0.5f * bs.y);
             float l0 = 1.f, l1 = 1.f;
 #pragma unroll
             for (int rr = 0; rr < 16; ++rr) {
@@ -361,7 +362,7 @@ __global__ void __launch_bounds__(NTHR, 1) kda_chunk_tc_kernel(KdaChunkArgs a) {
                     } else {
                         float ex = (fa ? 0.f : 0.5f * bsa) + (fb ? 0.f : 0.5f * bsb);
                         for (int j = pb + 1; j < pa; ++j) ex += sBS[j * 128 + ch];
-                        sc = expf(ex);
+                        sc = __expf(ex);
                     }
                     sSC[p * 128 + ch] = sc;
                 }
@@ -371,14 +372,6 @@ __global__ void __launch_bounds__(NTHR, 1) kda_chunk_tc_kernel(KdaChunkArgs a) {
         tc_fence_before();
         __syncthreads();
         tc_fence_after();
-        // q, k of the next chunk can now replace this chunk's; log_alpha and beta into registers.
-        if (ci + 1 < nchunks) {
-            const ChunkPos cn = chunk_pos(t0, t1, ci + 1);
-            issue_qk(sm, qg, kg, cn, H, h, tid);
-            load_la(la, a.log_alpha, cn, H, h, eb, c2);
-            beta_next = (tid < CH && tid < cn.nr) ? a.beta[(size_t)(cn.c0 + tid) * H + h] : 0.f;
-        }
-        asm volatile("cp.async.commit_group;" ::: "memory");
 
         // ---------------- AP: A and P
         if (fast) {
@@ -607,6 +600,15 @@ __global__ void __launch_bounds__(NTHR, 1) kda_chunk_tc_kernel(KdaChunkArgs a) {
                          idesc_bf16(128, 128, false, true), ks > 0);
             mma_commit(&bar_w);
         }
+        // While the tensor core works: q, k of the next chunk replace this chunk's (dead since
+        // E2), and its log_alpha and beta go to registers.
+        if (ci + 1 < nchunks) {
+            const ChunkPos cn = chunk_pos(t0, t1, ci + 1);
+            issue_qk(sm, qg, kg, cn, H, h, tid);
+            load_la(la, a.log_alpha, cn, H, h, eb, c2);
+            beta_next = (tid < CH && tid < cn.nr) ? a.beta[(size_t)(cn.c0 + tid) * H + h] : 0.f;
+        }
+        asm volatile("cp.async.commit_group;" ::: "memory");
         if (!mbar_wait(&bar_w, par, kWaitCycles)) s_abort = 1;
         tc_fence_after();
         //      [-W; s q gamma - P W] -> tensor-core operand (K-major, 2 x 128 lines)
