@@ -47,7 +47,7 @@ extern "C" int kda_chunk_fwd(const void *q, const void *k, const void *v, const 
                              void *out, float *S_final, int B, int T, int H, int dk, int dv, int C,
                              int dtype, kda_stream_t stream) {
     if (dtype != KDA_F32 && dtype != KDA_BF16) return KDA_ERR_DTYPE;
-    if (B < 1 || H < 1 || T < 0 || !dim_ok(dk) || !dim_ok(dv)) return KDA_ERR_DIM;
+    if (B < 1 || H < 1 || H > 65535 || T < 0 || !dim_ok(dk) || !dim_ok(dv)) return KDA_ERR_DIM;
     if (C != 64) return KDA_ERR_CHUNK;
     const int64_t T_total = cu_seqlens ? (int64_t)T : (int64_t)B * T;
     // Token tensors may be NULL only when there are no tokens at all.

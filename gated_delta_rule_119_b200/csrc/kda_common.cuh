@@ -63,4 +63,6 @@ cudaError_t kda_launch_chunk_simt_f32(const KdaChunkArgs &a, cudaStream_t stream
 cudaError_t kda_launch_chunk_simt_bf16(const KdaChunkArgs &a, cudaStream_t stream);
 cudaError_t kda_launch_chunk_tc(const KdaChunkArgs &a, cudaStream_t stream);
 bool kda_chunk_tc_supports(int dk, int dv);
+size_t kda_chunk_tc_workspace_bytes(const KdaChunkArgs &a);
+cudaError_t kda_launch_chunk_tc_ws(const KdaChunkArgs &a, void *ws, cudaStream_t stream);
 cudaError_t kda_read_device_status(unsigned int *status, bool clear);
