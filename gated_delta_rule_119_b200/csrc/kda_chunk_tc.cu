@@ -117,11 +117,34 @@ __global__ void kda_chunk_slots_kernel(const int32_t *cu_seqlens, int N, int64_t
     base[N] = acc;
 }
 
+// Exact diagonal-block contribution of one channel whose decay over a 16-row block is too
+// strong for the rescaled factors: running products of alpha, inputs re-read from memory.
+// Adds beta_r k_r k_i D_ri to A (i < r) and s q_r k_i D_ri to the block's exact P sums.
+__device__ __noinline__ void exact_diag_channel(const KdaChunkArgs &a, int64_t c0, int nr, int h, int blk,
+                                                int ch, const float *sBeta, float *Am, float *sCP) {
+    const int H = a.H;
+    const __nv_bfloat16 *qg = static_cast<const __nv_bfloat16 *>(a.q);
+    const __nv_bfloat16 *kg = static_cast<const __nv_bfloat16 *>(a.k);
+    for (int i = 0; i < 16; ++i) {
+        const int I = 16 * blk + i;
+        if (I >= nr) break;
+        const float ki = __bfloat162float(kg[((size_t)(c0 + I) * H + h) * DK + ch]);
+        float f = 1.f;
+        for (int R = I; R < 16 * blk + 16 && R < nr; ++R) {
+            const size_t off = ((size_t)(c0 + R) * H + h) * DK + ch;
+            if (R > I) f *= __expf(a.log_alpha[off]);
+            const float kd = ki * f;
+            if (R > I) atomicAdd(&Am[R * LF + I], sBeta[R] * __bfloat162float(kg[off]) * kd);
+            atomicAdd(&sCP[blk * 256 + (R - 16 * blk) * 16 + i], a.scale * __bfloat162float(qg[off]) * kd);
+        }
+    }
+}
+
 // ======================================================================= intra-chunk kernel
 __global__ void __launch_bounds__(NTHR, 2)
     kda_chunk_intra_kernel(KdaChunkArgs a, uint8_t *ws, const int32_t *slot_base) {
     extern __shared__ uint8_t smraw[];
-    uint8_t *sm = (uint8_t *)(((uintptr_t)smraw + 1023) & ~(uintptr_t)1023);
+    uint8_t *sm = smraw + ((1024u - (smem_u32(smraw) & 1023u)) & 1023u);   // stays a shared-space pointer
     __shared__ uint64_t bar_ap, bar_p, bar_w;
     __shared__ uint32_t s_tmem;
     __shared__ int s_abort;
@@ -163,7 +186,7 @@ __global__ void __launch_bounds__(NTHR, 2)
     // E2 thread mapping: channels {c2, c2 + 1} of 16-row block eb.  All loads up front.
     const int c2 = 2 * (tid & 63), eb = tid >> 6;
     float2 la[16];
-    uint32_t kr2[16], qr2[16];
+    uint32_t kr2[16];
 #pragma unroll
     for (int rr = 0; rr < 16; ++rr) {
         const int r = 16 * eb + rr;
@@ -171,7 +194,15 @@ __global__ void __launch_bounds__(NTHR, 2)
         const bool ok = r < nr;
         la[rr] = ok ? *reinterpret_cast<const float2 *>(a.log_alpha + off) : make_float2(0.f, 0.f);
         kr2[rr] = ok ? *reinterpret_cast<const uint32_t *>(kg + off) : 0u;
-        qr2[rr] = ok ? *reinterpret_cast<const uint32_t *>(qg + off) : 0u;
+    }
+    // q goes to shared memory (row-major [64][128] in the space of [T'; P T'], unused until
+    // then), which keeps it out of the registers; rows past the chunk's end are zero-filled.
+    uint8_t *sQ = sTP;
+#pragma unroll
+    for (int k4 = 0; k4 < 4; ++k4) {
+        const int idx = tid + NTHR * k4, r = idx >> 4, j = idx & 15;
+        const bool ok = r < nr;
+        cp_async16(sQ + r * 256 + 16 * j, ok ? qg + ((size_t)(c0 + r) * H + h) * DK + 8 * j : qg, ok ? 16u : 0u);
     }
     if (tid < CH) sBeta[tid] = tid < nr ? a.beta[(size_t)(c0 + tid) * H + h] : 0.f;
 
@@ -205,6 +236,7 @@ __global__ void __launch_bounds__(NTHR, 2)
         *reinterpret_cast<float2 *>(&sBS[eb * 128 + c2]) = make_float2(s0, s1);
         *reinterpret_cast<float2 *>(&sBT[eb * 128 + c2]) = make_float2(p0, p1);
     }
+    cp_async_wait_all();
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
@@ -242,55 +274,58 @@ __global__ void __launch_bounds__(NTHR, 2)
         const float rho1 = fast || fl1 ? 1.f : __expf(-0.5f * bs.y);
         __nv_bfloat16 *gKL = (__nv_bfloat16 *)(gslot + SLOT_KL), *gKR = (__nv_bfloat16 *)(gslot + SLOT_KR);
         __nv_bfloat16 *gQL = (__nv_bfloat16 *)(gslot + SLOT_QL);
-        float l0 = 1.f, l1 = 1.f;
+        if (fast) {
+            float l0 = 1.f, l1 = 1.f;
 #pragma unroll
-        for (int rr = 0; rr < 16; ++rr) {
-            const int r = 16 * eb + rr;
-            l0 *= la[rr].x;
-            l1 *= la[rr].y;
-            const float2 kv = unpack_bf16(kr2[rr]), qv = unpack_bf16(qr2[rr]);
-            const float g0 = gpre.x * l0, g1 = gpre.y * l1;
-            *(uint32_t *)(sKQ + col_kq + sw128(r, c2 & 63)) = pack_bf16(kv.x * g0, kv.y * g1);
-            *(uint32_t *)(sKQ + col_kq + sw128(64 + r, c2 & 63)) = pack_bf16(scale * qv.x * g0, scale * qv.y * g1);
-            if (!fast) {
+            for (int rr = 0; rr < 16; ++rr) {
+                const int r = 16 * eb + rr;
+                l0 *= la[rr].x;
+                l1 *= la[rr].y;
+                const float2 kv = unpack_bf16(kr2[rr]), qv = unpack_bf16(*(const uint32_t *)(sQ + r * 256 + 2 * c2));
+                const float g0 = gpre.x * l0, g1 = gpre.y * l1;
+                *(uint32_t *)(sKQ + col_kq + sw128(r, c2 & 63)) = pack_bf16(kv.x * g0, kv.y * g1);
+                *(uint32_t *)(sKQ + col_kq + sw128(64 + r, c2 & 63)) = pack_bf16(scale * qv.x * g0, scale * qv.y * g1);
+            }
+            float g0 = 1.f, g1 = 1.f;
+#pragma unroll
+            for (int rr = 15; rr >= 0; --rr) {
+                const int r = 16 * eb + rr;
+                const float2 kv = unpack_bf16(kr2[rr]);
+                const uint32_t kc = pack_bf16(kv.x * (g0 * ksuf.x), kv.y * (g1 * ksuf.y));
+                *(uint32_t *)(gslot + SLOT_KC + col_kc + sw128(r, c2 & 63)) = kc;
+                *(uint32_t *)(sKC + col_kc + sw128(r, c2 & 63)) = kc;
+                g0 *= la[rr].x;
+                g1 *= la[rr].y;
+            }
+        } else {
+            float l0 = 1.f, l1 = 1.f;
+#pragma unroll
+            for (int rr = 0; rr < 16; ++rr) {
+                const int r = 16 * eb + rr;
+                l0 *= la[rr].x;
+                l1 *= la[rr].y;
+                const float2 kv = unpack_bf16(kr2[rr]), qv = unpack_bf16(*(const uint32_t *)(sQ + r * 256 + 2 * c2));
+                const float g0 = gpre.x * l0, g1 = gpre.y * l1;
+                *(uint32_t *)(sKQ + col_kq + sw128(r, c2 & 63)) = pack_bf16(kv.x * g0, kv.y * g1);
+                *(uint32_t *)(sKQ + col_kq + sw128(64 + r, c2 & 63)) = pack_bf16(scale * qv.x * g0, scale * qv.y * g1);
                 *(uint32_t *)&gKL[r * 128 + c2] = pack_bf16(kv.x * (rho0 * l0), kv.y * (rho1 * l1));
                 *(uint32_t *)&gQL[r * 128 + c2] =
                     pack_bf16(scale * qv.x * (rho0 * l0), scale * qv.y * (rho1 * l1));
             }
-        }
-        float g0 = 1.f, g1 = 1.f;
+            float g0 = 1.f, g1 = 1.f;
 #pragma unroll
-        for (int rr = 15; rr >= 0; --rr) {
-            const int r = 16 * eb + rr;
-            const float2 kv = unpack_bf16(kr2[rr]);
-            const uint32_t kc = pack_bf16(kv.x * (g0 * ksuf.x), kv.y * (g1 * ksuf.y));
-            *(uint32_t *)(gslot + SLOT_KC + col_kc + sw128(r, c2 & 63)) = kc;
-            if (fast) *(uint32_t *)(sKC + col_kc + sw128(r, c2 & 63)) = kc;
-            else *(uint32_t *)&gKR[r * 128 + c2] = pack_bf16(kv.x * (rho0 * g0), kv.y * (rho1 * g1));
-            g0 *= la[rr].x;
-            g1 *= la[rr].y;
-        }
-        if (!fast && (fl0 || fl1)) {
-            // Exact diagonal-block contribution of a flagged channel (running products).
-#pragma unroll
-            for (int cc = 0; cc < 2; ++cc) {
-                if (!(cc ? fl1 : fl0)) continue;
-#pragma unroll
-                for (int i = 0; i < 16; ++i) {
-                    const float ki = cc ? unpack_bf16(kr2[i]).y : unpack_bf16(kr2[i]).x;
-                    float f = 1.f;
-#pragma unroll
-                    for (int r = i; r < 16; ++r) {
-                        if (r > i) f *= cc ? la[r].y : la[r].x;
-                        const float2 kv = unpack_bf16(kr2[r]), qv = unpack_bf16(qr2[r]);
-                        const float kd = ki * f;
-                        const int R = 16 * eb + r;
-                        if (r > i) atomicAdd(&Am[R * LF + 16 * eb + i], sBeta[R] * (cc ? kv.y : kv.x) * kd);
-                        atomicAdd(&sCP[eb * 256 + r * 16 + i], scale * (cc ? qv.y : qv.x) * kd);
-                    }
-                }
+            for (int rr = 15; rr >= 0; --rr) {
+                const int r = 16 * eb + rr;
+                const float2 kv = unpack_bf16(kr2[rr]);
+                *(uint32_t *)(gslot + SLOT_KC + col_kc + sw128(r, c2 & 63)) =
+                    pack_bf16(kv.x * (g0 * ksuf.x), kv.y * (g1 * ksuf.y));
+                *(uint32_t *)&gKR[r * 128 + c2] = pack_bf16(kv.x * (rho0 * g0), kv.y * (rho1 * g1));
+                g0 *= la[rr].x;
+                g1 *= la[rr].y;
             }
         }
+        if (!fast && fl0) exact_diag_channel(a, c0, nr, h, eb, c2, sBeta, Am, sCP);
+        if (!fast && fl1) exact_diag_channel(a, c0, nr, h, eb, c2 + 1, sBeta, Am, sCP);
         if (eb == 0) {
             float2 gc = make_float2(1.f, 1.f);
 #pragma unroll
@@ -369,7 +404,7 @@ __global__ void __launch_bounds__(NTHR, 2)
             const int mat = task / 10, p = task % 10, pa = kPairA[p], pb = kPairB[p];
             const __nv_bfloat16 *Ls = mat == 0 ? gKL : gQL;
             float acc[2][2][4] = {};
-#pragma unroll
+#pragma unroll 2
             for (int kt = 0; kt < 8; ++kt) {
                 const int c = 16 * kt + 2 * t4;
                 const uint32_t a0 = *(const uint32_t *)&Ls[(16 * pa + g) * 128 + c];
@@ -585,7 +620,7 @@ __global__ void __launch_bounds__(NTHR, 2)
 __global__ void __launch_bounds__(NTHR, 1)
     kda_chunk_scan_kernel(KdaChunkArgs a, const uint8_t *ws, const int32_t *slot_base) {
     extern __shared__ uint8_t smraw[];
-    uint8_t *sm = (uint8_t *)(((uintptr_t)smraw + 1023) & ~(uintptr_t)1023);
+    uint8_t *sm = smraw + ((1024u - (smem_u32(smraw) & 1023u)) & 1023u);   // stays a shared-space pointer
     __shared__ uint64_t bar_ld[2], bar_uo, bar_s;
     __shared__ uint32_t s_tmem;
     __shared__ int s_abort;
@@ -661,6 +696,17 @@ __global__ void __launch_bounds__(NTHR, 1)
         tmem_st32(T_S + lane_off + half * 32, v);
     }
 
+    // Matrix descriptors of both stages (start address in the low bits; see desc_sw128).
+    const uint64_t d_tp0 = desc_sw128(smem_u32(sm + SLOT_TP), 16, 1024);
+    const uint64_t d_tp1 = desc_sw128(smem_u32(sm + S_STAGE + SLOT_TP), 16, 1024);
+    const uint64_t d_a20 = desc_sw128(smem_u32(sm + SLOT_A2), 16, 1024);
+    const uint64_t d_a21 = desc_sw128(smem_u32(sm + S_STAGE + SLOT_A2), 16, 1024);
+    const uint64_t d_kc0 = desc_sw128(smem_u32(sm + SLOT_KC), 8192, 1024);
+    const uint64_t d_kc1 = desc_sw128(smem_u32(sm + S_STAGE + SLOT_KC), 8192, 1024);
+    const uint64_t d_v0 = desc_sw128(smem_u32(sm + S_V), 8192, 1024);
+    const uint64_t d_v1 = desc_sw128(smem_u32(sm + S_STAGE + S_V), 8192, 1024);
+    const uint64_t d_s = desc_sw128(smem_u32(sS), 16384, 1024);
+
     uint64_t *pending = nullptr;
     uint32_t pending_par = 0;
     for (int ci = 0; ci < nchunks; ++ci) {
@@ -703,19 +749,16 @@ __global__ void __launch_bounds__(NTHR, 1)
         __syncthreads();
         tc_fence_after();
 
-        // [u; o] = [T'; P T'] v + [-W; Q'] S
+        // [u; o] = [T'; P T'] v + [-W; Q'] S.  Descriptor start addresses advance in 16-byte
+        // units: +2 per 16 columns of a K-major line, +128 per 16 lines of an MN-major tile.
         if (tid == 0) {
             const uint32_t idesc = idesc_bf16(128, DVT, false, true);
-            const uint32_t tp = smem_u32(st + SLOT_TP), vv = smem_u32(st + S_V);
-            const uint32_t a2 = smem_u32(st + SLOT_A2), ss = smem_u32(sS);
+            const uint64_t dtp = par ? d_tp1 : d_tp0, dv = par ? d_v1 : d_v0, da2 = par ? d_a21 : d_a20;
 #pragma unroll
-            for (int ks = 0; ks < 4; ++ks)
-                mma_bf16(T_UO, desc_sw128(tp + 32 * ks, 16, 1024), desc_sw128(vv + 2048 * ks, 8192, 1024),
-                         idesc, ks > 0);
+            for (int ks = 0; ks < 4; ++ks) mma_bf16(T_UO, dtp + 2 * ks, dv + 128 * ks, idesc, ks > 0);
 #pragma unroll
             for (int ks = 0; ks < 8; ++ks)
-                mma_bf16(T_UO, desc_sw128(a2 + (ks >> 2) * 16384 + 32 * (ks & 3), 16, 1024),
-                         desc_sw128(ss + 2048 * ks, 16384, 1024), idesc, 1);
+                mma_bf16(T_UO, da2 + (ks >> 2) * 1024 + 2 * (ks & 3), d_s + 128 * ks, idesc, 1);
             mma_commit(&bar_uo);
         }
         if (!mbar_wait(&bar_uo, par, kWaitCycles)) s_abort = 1;
@@ -744,11 +787,10 @@ __global__ void __launch_bounds__(NTHR, 1)
 
         // S += (update operand)^T u
         if (tid == 0) {
-            const uint32_t kc = smem_u32(st + SLOT_KC), uu = smem_u32(st + S_V);
+            const uint64_t dkc = par ? d_kc1 : d_kc0, du = par ? d_v1 : d_v0;
 #pragma unroll
             for (int ks = 0; ks < 4; ++ks)
-                mma_bf16(T_S, desc_sw128(kc + 2048 * ks, 8192, 1024), desc_sw128(uu + 2048 * ks, 8192, 1024),
-                         idesc_bf16(128, DVT, true, true), 1);
+                mma_bf16(T_S, dkc + 128 * ks, du + 128 * ks, idesc_bf16(128, DVT, true, true), 1);
             mma_commit(&bar_s);
         }
         if (!mbar_wait(&bar_s, par, kWaitCycles)) s_abort = 1;
