@@ -18,7 +18,8 @@
  * Conventions for every entry point:
  *  - All tensor arguments are DEVICE pointers on the current CUDA device, row-major,
  *    contiguous, 16-byte aligned.  The caller allocates and owns every buffer; the
- *    library keeps no pointer after a call returns and allocates no device memory.
+ *    library keeps no pointer after a call returns.  The only device memory the
+ *    library takes itself is kda_chunk_fwd's workspace (below).
  *  - Calls are asynchronous on `stream` (a cudaStream_t; NULL = legacy default
  *    stream) and never synchronise the device.
  *  - The return value is KDA_OK (0) or a negative kda_status.  Argument errors are
@@ -83,6 +84,13 @@ enum kda_status {
  *                                                 pointer as S0 (updated in place).
  *   C          chunk length; must be 64.
  * Empty sequences (and T = 0) are allowed: their S_final is S0 (or zero).
+ * Workspace: with KDA_BF16 and dk = dv = 128 the call runs two kernels (one per
+ * (chunk, head), then one scan per (sequence, head)) that hand each chunk's operands
+ * over through a device workspace of 66,560 bytes per (chunk, head) plus 4 (N + 1)
+ * bytes, rounded up to 1 KiB.  It is taken with cudaMallocAsync on `stream` from the
+ * device's default memory pool and returned with cudaFreeAsync on the same stream;
+ * the pool's release threshold is raised on first use so the memory stays in the
+ * pool between calls.  Every other dtype and size allocates nothing.
  * Supported sizes: KDA_F32 any dk, dv in {32, 64, 128}; KDA_BF16 dk = dv = 128, or
  * dk, dv in {32, 64, 128} through the same path.
  * q, k, v, log_alpha, beta and out may be NULL only when T_total = 0.
