@@ -15,8 +15,10 @@ LIB_PATH = os.path.join(HERE, "libkda.so")
 KDA_F32, KDA_BF16 = 0, 1
 STATUS = {0: "KDA_OK", -1: "KDA_ERR_NULL", -2: "KDA_ERR_DIM", -3: "KDA_ERR_CHUNK",
           -4: "KDA_ERR_ALIGN", -5: "KDA_ERR_DTYPE", -6: "KDA_ERR_ALIAS", -7: "KDA_ERR_CUDA",
-          -8: "KDA_ERR_TIMEOUT"}
-EXPORTS = ("kda_chunk_fwd", "kda_decode_step", "kda_device_status", "kda_status_string")
+          -8: "KDA_ERR_TIMEOUT", -9: "KDA_ERR_SCRATCH"}
+EXPORTS = ("kda_chunk_fwd", "kda_chunk_fwd_noalloc", "kda_decode_step", "kda_device_status",
+           "kda_status_string")
+NOALLOC_SCRATCH_BYTES = 64 * 1024 * 1024   # KDA_NOALLOC_SCRATCH_BYTES
 
 _lib = None
 
@@ -40,6 +42,8 @@ def load_library(path: str | None = None):
     V, F, I32 = ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int
     lib.kda_chunk_fwd.argtypes = [V, V, V, F, F, F, V, V, F] + [I32] * 7 + [V]
     lib.kda_chunk_fwd.restype = ctypes.c_int
+    lib.kda_chunk_fwd_noalloc.argtypes = [V, V, V, F, F, F, V, V, F] + [I32] * 7 + [V]
+    lib.kda_chunk_fwd_noalloc.restype = ctypes.c_int
     lib.kda_decode_step.argtypes = [V, V, V, F, F, F, V] + [I32] * 5 + [V]
     lib.kda_decode_step.restype = ctypes.c_int
     lib.kda_device_status.argtypes = []
@@ -69,6 +73,15 @@ def chunk_fwd_raw(q, k, v, log_alpha, beta, S0, cu_seqlens, out, S_final, B, T, 
                                         beta or None, S0 or None, cu_seqlens or None,
                                         out or None, S_final or None, B, T, H, dk, dv, C,
                                         dtype, stream or None)
+
+
+def chunk_fwd_noalloc_raw(q, k, v, log_alpha, beta, S0, cu_seqlens, out, S_final, B, T, H, dk,
+                          dv, C, dtype, stream) -> int:
+    """kda_chunk_fwd_noalloc with integer addresses (0 = NULL)."""
+    return load_library().kda_chunk_fwd_noalloc(q or None, k or None, v or None,
+                                                log_alpha or None, beta or None, S0 or None,
+                                                cu_seqlens or None, out or None, S_final or None,
+                                                B, T, H, dk, dv, C, dtype, stream or None)
 
 
 def decode_step_raw(q, k, v, log_alpha, beta, S_inout, out, N, H, dk, dv, dtype,

@@ -38,14 +38,20 @@ extern "C" const char *kda_status_string(int status) {
     case KDA_ERR_ALIAS: return "KDA_ERR_ALIAS: an output overlaps an input";
     case KDA_ERR_CUDA: return g_cuda_msg;
     case KDA_ERR_TIMEOUT: return "KDA_ERR_TIMEOUT: a bounded device-side wait gave up";
+    case KDA_ERR_SCRATCH:
+        return "KDA_ERR_SCRATCH: the problem needs more workspace than the fixed scratch buffer of "
+               "kda_chunk_fwd_noalloc holds (KDA_NOALLOC_SCRATCH_BYTES)";
     default: return "unknown kda status";
     }
 }
 
-extern "C" int kda_chunk_fwd(const void *q, const void *k, const void *v, const float *log_alpha,
-                             const float *beta, const float *S0, const int32_t *cu_seqlens,
-                             void *out, float *S_final, int B, int T, int H, int dk, int dv, int C,
-                             int dtype, kda_stream_t stream) {
+namespace {
+
+// Host-side checks of a chunked-prefill call; on success fills `a`.
+int prepare_chunk(const void *q, const void *k, const void *v, const float *log_alpha,
+                  const float *beta, const float *S0, const int32_t *cu_seqlens, void *out,
+                  float *S_final, int B, int T, int H, int dk, int dv, int C, int dtype,
+                  KdaChunkArgs &a) {
     if (dtype != KDA_F32 && dtype != KDA_BF16) return KDA_ERR_DTYPE;
     if (B < 1 || H < 1 || H > 65535 || T < 0 || !dim_ok(dk) || !dim_ok(dv)) return KDA_ERR_DIM;
     if (C != 64) return KDA_ERR_CHUNK;
@@ -72,10 +78,47 @@ extern "C" int kda_chunk_fwd(const void *q, const void *k, const void *v, const 
     if (S0 && S_final && overlap(in_s0, sf) && (const void *)S0 != (const void *)S_final)
         return KDA_ERR_ALIAS;
 
-    KdaChunkArgs a{q, k, v, log_alpha, beta, S0, cu_seqlens, out, S_final, B, T, H, dk, dv,
-                   T_total, 1.0f / sqrtf((float)dk)};
+    a = KdaChunkArgs{q, k, v, log_alpha, beta, S0, cu_seqlens, out, S_final, B, T, H, dk, dv,
+                     T_total, 1.0f / sqrtf((float)dk)};
+    return KDA_OK;
+}
+
+}  // namespace
+
+extern "C" int kda_chunk_fwd(const void *q, const void *k, const void *v, const float *log_alpha,
+                             const float *beta, const float *S0, const int32_t *cu_seqlens,
+                             void *out, float *S_final, int B, int T, int H, int dk, int dv, int C,
+                             int dtype, kda_stream_t stream) {
+    KdaChunkArgs a;
+    const int rc = prepare_chunk(q, k, v, log_alpha, beta, S0, cu_seqlens, out, S_final, B, T, H,
+                                 dk, dv, C, dtype, a);
+    if (rc != KDA_OK) return rc;
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
     if (dtype == KDA_BF16 && kda_chunk_tc_supports(dk, dv)) return cuda_status(kda_launch_chunk_tc(a, st));
+    return cuda_status(dtype == KDA_F32 ? kda_launch_chunk_simt_f32(a, st)
+                                        : kda_launch_chunk_simt_bf16(a, st));
+}
+
+// The same computation as kda_chunk_fwd with no device allocation: the tensor-core
+// path's workspace is the library's fixed per-device scratch buffer; the other paths
+// need none.  The size check runs on the host before any CUDA call.
+extern "C" int kda_chunk_fwd_noalloc(const void *q, const void *k, const void *v,
+                                     const float *log_alpha, const float *beta, const float *S0,
+                                     const int32_t *cu_seqlens, void *out, float *S_final, int B,
+                                     int T, int H, int dk, int dv, int C, int dtype,
+                                     kda_stream_t stream) {
+    KdaChunkArgs a;
+    const int rc = prepare_chunk(q, k, v, log_alpha, beta, S0, cu_seqlens, out, S_final, B, T, H,
+                                 dk, dv, C, dtype, a);
+    if (rc != KDA_OK) return rc;
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    if (dtype == KDA_BF16 && kda_chunk_tc_supports(dk, dv)) {
+        if (kda_chunk_tc_workspace_bytes(a) > (size_t)KDA_NOALLOC_SCRATCH_BYTES) return KDA_ERR_SCRATCH;
+        void *scratch = nullptr;
+        const cudaError_t e = kda_noalloc_scratch(&scratch);
+        if (e != cudaSuccess) return cuda_status(e);
+        return cuda_status(kda_launch_chunk_tc_ws(a, scratch, st));
+    }
     return cuda_status(dtype == KDA_F32 ? kda_launch_chunk_simt_f32(a, st)
                                         : kda_launch_chunk_simt_bf16(a, st));
 }

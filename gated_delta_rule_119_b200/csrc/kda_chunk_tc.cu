@@ -827,14 +827,23 @@ cudaError_t configure(int dev) {
     if (e != cudaSuccess) return e;
     e = cudaFuncSetAttribute(kda_chunk_scan_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kScanSmem);
     if (e != cudaSuccess) return e;
-    // Keep freed workspace in the pool between calls instead of returning it to the driver.
+    if (dev >= 0 && dev < 64) g_configured[dev] = true;
+    return cudaSuccess;
+}
+
+bool g_pool_configured[64] = {};
+
+// Keep freed workspace in the device's default pool between calls instead of returning
+// it to the driver.
+cudaError_t configure_pool(int dev) {
+    if (dev >= 0 && dev < 64 && g_pool_configured[dev]) return cudaSuccess;
     cudaMemPool_t pool;
-    e = cudaDeviceGetDefaultMemPool(&pool, dev);
+    cudaError_t e = cudaDeviceGetDefaultMemPool(&pool, dev);
     if (e != cudaSuccess) return e;
     uint64_t keep = ~0ull;
     e = cudaMemPoolSetAttribute(pool, cudaMemPoolAttrReleaseThreshold, &keep);
     if (e != cudaSuccess) return e;
-    if (dev >= 0 && dev < 64) g_configured[dev] = true;
+    if (dev >= 0 && dev < 64) g_pool_configured[dev] = true;
     return cudaSuccess;
 }
 
@@ -876,6 +885,7 @@ cudaError_t kda_launch_chunk_tc(const KdaChunkArgs &a, cudaStream_t stream) {
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return e;
     if ((e = configure(dev)) != cudaSuccess) return e;
+    if ((e = configure_pool(dev)) != cudaSuccess) return e;
     void *ws = nullptr;
     if ((e = cudaMallocAsync(&ws, kda_chunk_tc_workspace_bytes(a), stream)) != cudaSuccess) return e;
     e = kda_launch_chunk_tc_ws(a, ws, stream);

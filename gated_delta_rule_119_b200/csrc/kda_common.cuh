@@ -65,4 +65,6 @@ cudaError_t kda_launch_chunk_tc(const KdaChunkArgs &a, cudaStream_t stream);
 bool kda_chunk_tc_supports(int dk, int dv);
 size_t kda_chunk_tc_workspace_bytes(const KdaChunkArgs &a);
 cudaError_t kda_launch_chunk_tc_ws(const KdaChunkArgs &a, void *ws, cudaStream_t stream);
+// Device address of the fixed scratch buffer of the current device (kda_noalloc.cu).
+cudaError_t kda_noalloc_scratch(void **ptr);
 cudaError_t kda_read_device_status(unsigned int *status, bool clear);

@@ -19,7 +19,8 @@
  *  - All tensor arguments are DEVICE pointers on the current CUDA device, row-major,
  *    contiguous, 16-byte aligned.  The caller allocates and owns every buffer; the
  *    library keeps no pointer after a call returns.  The only device memory the
- *    library takes itself is kda_chunk_fwd's workspace (below).
+ *    library takes itself is kda_chunk_fwd's workspace (below); kda_chunk_fwd_noalloc
+ *    uses a fixed buffer instead.
  *  - Calls are asynchronous on `stream` (a cudaStream_t; NULL = legacy default
  *    stream) and never synchronise the device.
  *  - The return value is KDA_OK (0) or a negative kda_status.  Argument errors are
@@ -58,7 +59,8 @@ enum kda_status {
     KDA_ERR_DTYPE = -5,   /* dtype is not a kda_dtype */
     KDA_ERR_ALIAS = -6,   /* an output overlaps an input it must not overlap */
     KDA_ERR_CUDA = -7,    /* a CUDA launch failed; kda_status_string names the CUDA error */
-    KDA_ERR_TIMEOUT = -8  /* reserved for bounded device-side waits */
+    KDA_ERR_TIMEOUT = -8, /* reserved for bounded device-side waits */
+    KDA_ERR_SCRATCH = -9  /* kda_chunk_fwd_noalloc: the workspace would exceed its fixed buffer */
 };
 
 /*
@@ -102,6 +104,39 @@ int kda_chunk_fwd(const void *q, const void *k, const void *v, const float *log_
                   const float *beta, const float *S0, const int32_t *cu_seqlens, void *out,
                   float *S_final, int B, int T, int H, int dk, int dv, int C, int dtype,
                   kda_stream_t stream);
+
+/*
+ * kda_chunk_fwd_noalloc -- kda_chunk_fwd that takes no device memory.
+ *
+ * The pages have no counterpart of this call: it adds nothing to the method.  It is
+ * for callers that must not allocate during a call -- a server that reserved nearly
+ * all of HBM for its caches at start-up, a runtime whose device footprint must be
+ * fixed in advance, a host thread that must keep clear of allocator state.
+ * Arguments, layouts, results and errors are those of kda_chunk_fwd, plus
+ * KDA_ERR_SCRATCH.  Where kda_chunk_fwd takes its workspace from the memory pool,
+ * this call uses a buffer of KDA_NOALLOC_SCRATCH_BYTES (64 MiB) that is part of the
+ * library's device image, one per device; no allocator (CUDA's or any other) is called.
+ *  - Limit: the workspace must fit: 66,560 bytes per (chunk, head) plus 4 (N + 1)
+ *    bytes rounded up to 1 KiB, counting ceil(T / 64) chunks per sequence without
+ *    cu_seqlens and ceil(T / 64) + N chunks in all with it.  That is at most 1,008
+ *    (chunk, head) pairs, e.g. one 4,032-token sequence with 16 heads.  A larger
+ *    problem returns KDA_ERR_SCRATCH, found on the host before any CUDA call.  Only
+ *    KDA_BF16 with dk = dv = 128 uses the buffer; every other case needs none.
+ *  - The first call on a device looks up the buffer's device address (one CUDA runtime
+ *    query, made with that device current) and keeps it.  A caller that records its
+ *    calls into a stream capture should make one call on each device before it starts.
+ *  - Nothing in the buffer needs to start at zero: each call writes every byte of it
+ *    that the call later reads.
+ *  - Overlapping calls race: two calls on one device that can run at the same time
+ *    (different streams, or host threads with no ordering between their streams)
+ *    share the buffer and corrupt each other's results.  Calls on one stream are
+ *    ordered and safe.
+ */
+#define KDA_NOALLOC_SCRATCH_BYTES (64u * 1024u * 1024u)
+int kda_chunk_fwd_noalloc(const void *q, const void *k, const void *v, const float *log_alpha,
+                          const float *beta, const float *S0, const int32_t *cu_seqlens,
+                          void *out, float *S_final, int B, int T, int H, int dk, int dv, int C,
+                          int dtype, kda_stream_t stream);
 
 /*
  * kda_decode_step -- one recurrent step (one new token) for N independent sequences.
