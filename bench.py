@@ -160,8 +160,9 @@ def source_digest(rel: str) -> str:
 
 
 def profiled_traffic(kernel_key: str, workload: str):
-    """DRAM bytes per launch recorded in a committed ncu summary, or None when
-    there is none or the kernel source changed since it was taken."""
+    """DRAM bytes per call recorded in a committed ncu summary (for the tensor-core
+    prefill: both of its kernels, read + write), or None when there is none or the
+    kernel source changed since it was taken."""
     stem = os.path.splitext(os.path.basename(KERNEL_SOURCES[kernel_key]))[0]
     path = os.path.join(PROFILES, f"{stem}__{workload}.md")
     if not os.path.exists(path):
@@ -260,7 +261,7 @@ def run_ours(args, rank, local_rank, world):
     hbm, bf16_tf, peak_kind = measured_peaks()
     stream = torch.cuda.current_stream(device)
     es = 2 if w["dtype"] == "bf16" else 4
-    launches_per_step = 1
+    launches_per_step = 1        # decode: one kernel; SIMT prefill: one kernel
 
     if name == "decode":
         N, H, dk, dv = w["B"], w["H"], w["dk"], w["dv"]
@@ -298,6 +299,9 @@ def run_ours(args, rank, local_rank, world):
         flops_per_launch = alg_flops_prefill(tok_heads, inp.dk, inp.dv)
         kernel_key = "chunk" if (w["dtype"] == "bf16" and w["dk"] == 128 and w["dv"] == 128) \
             else "chunk_simt"
+        if kernel_key == "chunk":
+            # intra-chunk kernel + scan kernel, plus the slot-offset kernel for varlen
+            launches_per_step = 2 + (inp.cu_seqlens is not None)
         inp_for_cpu = inp
 
     for i in range(args.warmup):
@@ -317,7 +321,10 @@ def run_ours(args, rank, local_rank, world):
     ms_local = ev0.elapsed_time(ev1) / args.steps
     ms = reduce_max(ms_local, device)
 
-    # per-launch duration of the dominant (only) kernel, events around each launch
+    # Duration of one call, events around each call on the launching stream.  For the
+    # tensor-core prefill a call is its two kernels back to back (intra-chunk, then
+    # scan); the roofline is taken over the call because the algorithmic bytes (q, k,
+    # v, gates in; o and states out) belong to the pair, not to either kernel alone.
     evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
            for _ in range(min(args.steps, 20))]
     for i, (a, b) in enumerate(evs):
@@ -346,8 +353,11 @@ def run_ours(args, rank, local_rank, world):
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": hbm, "unit": "GB/s",
                      "frac": achieved / hbm, "traffic": traffic,
                      "peak_kind": f"{peak_kind} (STREAM-style copy, burst)",
-                     "kernel": kernel_key, "alg_bytes_per_launch": bytes_per_launch,
-                     "launch_ms": launch_ms},
+                     "kernel": {"chunk": "kda_chunk_intra_kernel + kda_chunk_scan_kernel "
+                                          "(one kda_chunk_fwd call)",
+                                "chunk_simt": "kda_chunk_simt_kernel",
+                                "decode": "kda_decode_kernel"}[kernel_key],
+                     "alg_bytes_per_launch": bytes_per_launch, "launch_ms": launch_ms},
         "clocks": clk.summary(),
         "e2e": e2e,
         "gpu_launches": args.steps * launches_per_step,
@@ -385,17 +395,18 @@ def run_e2e(args, name, device, stream, rank):
         S_host = torch.empty((inp.n_seqs, inp.H, inp.dk, inp.dv), dtype=torch.float32).pin_memory()
         units = inp.total_tokens
     h2d = sum(t.numel() * t.element_size() for t in host.values() if t is not None)
+    # Decode keeps the recurrent state resident in HBM across steps (it is the model's
+    # memory, not a step input): a step moves the new token's q, k, v and gates in and
+    # its o out.  Prefill moves every input in and o plus the final states out.
+    d2h = out_host.numel() * out_host.element_size() + (0 if name == "decode" else S_host.numel() * 4)
     if name == "decode":
-        h2d += S_host.numel() * 4
-    d2h = out_host.numel() * out_host.element_size() + S_host.numel() * 4
+        S_dev.copy_(S_host)
 
     def one():
         d = {k: (None if t is None else t.to(device, non_blocking=True)) for k, t in host.items()}
         if name == "decode":
-            S_dev.copy_(S_host, non_blocking=True)
             o = kda_decode_step(d["q"], d["k"], d["v"], d["log_alpha"], d["beta"], S_dev)
             out_host.copy_(o, non_blocking=True)
-            S_host.copy_(S_dev, non_blocking=True)
         else:
             o, Sf = kda_chunk_fwd(d["q"], d["k"], d["v"], d["log_alpha"], d["beta"], d["S0"],
                                   d["cu_seqlens"])
@@ -415,7 +426,8 @@ def run_e2e(args, name, device, stream, rank):
     world = int(os.environ.get("WORLD_SIZE", 1))
     return {"value": units * world / (ms / 1e3), "unit": "tokens/s", "ms_per_step": ms,
             "steps": steps, "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
-            "path": "pinned host -> kda_* public call -> pinned host"}
+            "path": "pinned host -> kda_* public call -> pinned host"
+                    + (" (decode state resident in HBM)" if name == "decode" else "")}
 
 
 def run_reference(args, rank, world):
