@@ -34,7 +34,10 @@
 //      update operand k kappa.
 //  T   T = (I + A)^{-1}: 16 x 16 diagonal blocks by substitution in fp32, the rest with
 //      tf32 warp MMAs; [T'; P T'] = [I; P] T' and [W; P W] = [T'; P T'] (k gamma) on tcgen05.
+#include <cuda.h>
+#include <cudaTypedefs.h>
 #include <stdio.h>
+#include <string.h>
 
 #include "kda_common.cuh"
 #include "kda_tc_util.cuh"
@@ -81,6 +84,7 @@ constexpr uint32_t I_END = I_XT + 3072;
 constexpr size_t kIntraSmem = I_END + 1024;
 static_assert(I_TP % 1024 == 0 && I_KC % 1024 == 0, "tile alignment");
 static_assert(I_CP + 4096 <= I_TP, "block-path scratch inside T");
+static_assert(I_AM + 32768 <= I_TP, "[-W; s q gamma - P W] staged in the space of A and T");
 static_assert(2 * (kIntraSmem + 1024) <= 233472, "two intra CTAs per SM");
 
 // Scan kernel shared memory: two stages of {slot image, v slice}, the bf16 state copy.
@@ -291,9 +295,8 @@ __global__ void __launch_bounds__(NTHR, 2)
             for (int rr = 15; rr >= 0; --rr) {
                 const int r = 16 * eb + rr;
                 const float2 kv = unpack_bf16(kr2[rr]);
-                const uint32_t kc = pack_bf16(kv.x * (g0 * ksuf.x), kv.y * (g1 * ksuf.y));
-                *(uint32_t *)(gslot + SLOT_KC + col_kc + sw128(r, c2 & 63)) = kc;
-                *(uint32_t *)(sKC + col_kc + sw128(r, c2 & 63)) = kc;
+                *(uint32_t *)(sKC + col_kc + sw128(r, c2 & 63)) =
+                    pack_bf16(kv.x * (g0 * ksuf.x), kv.y * (g1 * ksuf.y));
                 g0 *= la[rr].x;
                 g1 *= la[rr].y;
             }
@@ -364,6 +367,8 @@ __global__ void __launch_bounds__(NTHR, 2)
     // ---------------- AP: A (fp32, to Am) and P (bf16, lines 64-127 of [I; P])
     if (fast) {
         if (tid == 0) {
+            bulk_s2g(gslot + SLOT_KC, sKC, 16384);      // the update operand, already in slot layout
+            bulk_commit();
             const uint32_t kq = smem_u32(sKQ), kc = smem_u32(sKC);
 #pragma unroll
             for (int ks = 0; ks < 8; ++ks)
@@ -377,7 +382,8 @@ __global__ void __launch_bounds__(NTHR, 2)
         float v[32];
         tmem_ld32(T_AP + lane_off + half * 32, v);
         tc_fence_before();
-        __syncthreads();   // the product has consumed k e^-g: its space becomes [I; P]
+        if (tid == 0) bulk_wait_read_all();
+        __syncthreads();   // the product and the bulk store have read k e^-g: its space becomes [I; P]
         const int r = trow & 63;
         if (trow < 64) {
             const float bb = sBeta[r];
@@ -578,14 +584,15 @@ __global__ void __launch_bounds__(NTHR, 2)
                      idesc_bf16(128, 128, false, true), ks > 0);
         mma_commit(&bar_w);
     }
-#pragma unroll
-    for (int k4 = 0; k4 < 4; ++k4) {
-        const int o = tid + NTHR * k4;
-        *(uint4 *)(gslot + SLOT_TP + 16 * o) = *(const uint4 *)(sTP + 16 * o);
+    if (tid == 32) {
+        bulk_s2g(gslot + SLOT_TP, sTP, 16384);
+        bulk_commit();
     }
     if (!mbar_wait(&bar_w, 0, kWaitCycles)) s_abort = 1;
     tc_fence_after();
-    //      [-W; s q gamma - P W] -> the slot (K-major, 2 x 128 lines)
+    //      [-W; s q gamma - P W] -> shared memory in the slot's layout (K-major, 2 x 128 lines;
+    //      the space of A and T, no longer needed), then one bulk store to the slot
+    uint8_t *sA2 = sm + I_AM;
 #pragma unroll
     for (int part = 0; part < 2; ++part) {
         float v[32];
@@ -608,28 +615,52 @@ __global__ void __launch_bounds__(NTHR, 2)
         }
 #pragma unroll
         for (int m = 0; m < 4; ++m)
-            *(uint4 *)(gslot + SLOT_A2 + half * 16384 + sw128_chunk(trow, 4 * part + m)) = pack8(v + 8 * m);
+            *(uint4 *)(sA2 + half * 16384 + sw128_chunk(trow, 4 * part + m)) = pack8(v + 8 * m);
     }
-    if (s_abort && tid == 0) atomicOr(&g_kda_device_status, 1u);
+    fence_async_smem();
     tc_fence_before();
+    __syncthreads();
+    if (tid == 0) {
+        bulk_s2g(gslot + SLOT_A2, sA2, 32768);
+        bulk_commit();
+        bulk_wait_read_all();
+    }
+    if (tid == 32) bulk_wait_read_all();
+    if (s_abort && tid == 0) atomicOr(&g_kda_device_status, 1u);
     __syncthreads();
     if (warp == 0) tmem_free(tmem, 256);
 }
 
 // ============================================================================ scan kernel
-__global__ void __launch_bounds__(NTHR, 1)
-    kda_chunk_scan_kernel(KdaChunkArgs a, const uint8_t *ws, const int32_t *slot_base) {
+// One CTA per (sequence, head, 64-column d_v tile); the state tile S (128 x 64 fp32) stays in
+// TMEM for the whole sequence.  Warp roles, joined only through mbarriers:
+//   warps 0-7  read-out: per chunk c, S out of TMEM (pending decay applied, bf16 copy for the
+//              product), then [u; o] out of TMEM: u into shared memory (warps 0, 1, 4, 5 hold
+//              TMEM lanes 0-63), o to HBM (warps 2, 3, 6, 7);
+//   warp 8     tensor-core issue (one thread): [u; o] = [T'; P T'] v as soon as the chunk is in
+//              shared memory, + [-W; s q gamma - P W] S once S is copied, S += KC^T u once u is;
+//   warp 9     loads (one thread): slot c and the v tile of chunk c into stage c & 1 once the
+//              state product of chunk c - 2 has released it.
+// [u; o] alternates between two TMEM accumulators so chunk c + 1's first product can start
+// while o of chunk c is still being read.
+constexpr int SCAN_THREADS = 320;
+constexpr int kReadoutThreads = 256;
+
+__global__ void __launch_bounds__(SCAN_THREADS, 1)
+    kda_chunk_scan_kernel(KdaChunkArgs a, const uint8_t *ws, const int32_t *slot_base,
+                          const __grid_constant__ CUtensorMap tmap_v) {
     extern __shared__ uint8_t smraw[];
     uint8_t *sm = smraw + ((1024u - (smem_u32(smraw) & 1023u)) & 1023u);   // stays a shared-space pointer
-    __shared__ uint64_t bar_ld[2], bar_uo, bar_s;
+    __shared__ uint64_t bar_ld[2], bar_free[2], bar_ofree[2], bar_sready, bar_uo, bar_uready, bar_s;
     __shared__ uint32_t s_tmem;
-    __shared__ int s_abort;
+    __shared__ volatile int s_abort;
+    __shared__ int s_last, s_issued;      // last commit of the issuing thread (0 none, 1 uo, 2 s); loads issued
+    __shared__ uint32_t s_last_par;
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int H = a.H;
     const int pair = blockIdx.x / NTILE, tile = blockIdx.x % NTILE;
     const int n = pair / H, h = pair % H;
-    const __nv_bfloat16 *vg = static_cast<const __nv_bfloat16 *>(a.v);
     __nv_bfloat16 *og = static_cast<__nv_bfloat16 *>(a.out);
     int64_t t0, t1;
     kda::seq_bounds(a.cu_seqlens, n, a.T, a.T_total, t0, t1);
@@ -637,50 +668,35 @@ __global__ void __launch_bounds__(NTHR, 1)
     const int base = slot_base ? slot_base[n] : n * ((a.T + CH - 1) / CH);
     uint8_t *sS = sm + S_S;
 
-    // Bulk copy of slot `ci` (one thread, counted on bar_ld) and its v slice (cp.async).
-    auto issue_loads = [&](int ci) {
-        uint8_t *st = sm + (ci & 1) * S_STAGE;
-        if (tid == 0) {
-            const uint8_t *src = ws + ((size_t)(base + ci) * H + h) * SLOT_BYTES;
-            mbar_arrive_expect_tx(&bar_ld[ci & 1], SLOT_BYTES);
-#pragma unroll
-            for (int part = 0; part < 4; ++part)
-                bulk_g2s(st + part * (SLOT_BYTES / 4), src + part * (SLOT_BYTES / 4), SLOT_BYTES / 4,
-                         &bar_ld[ci & 1]);
-        }
-        const int64_t c0 = t0 + (int64_t)ci * CH;
-        const int nr = (int)(t1 - c0 < CH ? t1 - c0 : CH);
-        for (int idx = tid; idx < 512; idx += NTHR) {
-            const int r = idx >> 3, j = idx & 7;
-            const int rs = r < nr ? r : nr - 1;
-            cp_async16(st + S_V + sw128_chunk(r, j), vg + ((size_t)(c0 + rs) * H + h) * DV + tile * DVT + j * 8,
-                       r < nr ? 16u : 0u);
-        }
-        asm volatile("cp.async.commit_group;" ::: "memory");
-    };
-
     if (tid == 0) {
-        mbar_init(&bar_ld[0], 1);
-        mbar_init(&bar_ld[1], 1);
+        for (int i = 0; i < 2; ++i) {
+            mbar_init(&bar_ld[i], 1);
+            mbar_init(&bar_free[i], 1);
+            mbar_init(&bar_ofree[i], 4);
+        }
+        mbar_init(&bar_sready, 8);
         mbar_init(&bar_uo, 1);
+        mbar_init(&bar_uready, 4);
         mbar_init(&bar_s, 1);
         mbar_init_fence();
         s_abort = 0;
+        s_last = 0;
+        s_last_par = 0;
+        s_issued = 0;
     }
-    if (warp == 0) tmem_alloc(&s_tmem, 128);
-    tc_fence_before();
-    __syncthreads();
-    tc_fence_after();
-    if (nchunks > 0) issue_loads(0);
-    const uint32_t tmem = s_tmem, T_S = tmem, T_UO = tmem + DVT;
-    const int quarter = warp & 3, half = warp >> 2;
+    if (warp == 0) tmem_alloc(&s_tmem, 256);
+    const int quarter = warp & 3, half = (warp >> 2) & 1;
     const uint32_t lane_off = (uint32_t)(32 * quarter) << 16;
     const int trow = 32 * quarter + lane;
     const size_t s_base = ((size_t)pair * DK) * DV + (size_t)tile * DVT + half * 32;
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = s_tmem, T_S = tmem;          // [u; o] of chunk c: tmem + 64 + 64 (c & 1)
     // The state row trow is held in TMEM as S / pend: a fast-path chunk's decay is applied
     // when the state is next read.
     float pend = 1.f;
-    {
+    if (tid < kReadoutThreads) {
         float v[32];
         if (a.S0) {
             const float4 *src = reinterpret_cast<const float4 *>(a.S0 + s_base + (size_t)trow * DV);
@@ -695,117 +711,162 @@ __global__ void __launch_bounds__(NTHR, 1)
         }
         tmem_st32(T_S + lane_off + half * 32, v);
     }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
 
-    // Matrix descriptors of both stages (start address in the low bits; see desc_sw128).
-    const uint64_t d_tp0 = desc_sw128(smem_u32(sm + SLOT_TP), 16, 1024);
-    const uint64_t d_tp1 = desc_sw128(smem_u32(sm + S_STAGE + SLOT_TP), 16, 1024);
-    const uint64_t d_a20 = desc_sw128(smem_u32(sm + SLOT_A2), 16, 1024);
-    const uint64_t d_a21 = desc_sw128(smem_u32(sm + S_STAGE + SLOT_A2), 16, 1024);
-    const uint64_t d_kc0 = desc_sw128(smem_u32(sm + SLOT_KC), 8192, 1024);
-    const uint64_t d_kc1 = desc_sw128(smem_u32(sm + S_STAGE + SLOT_KC), 8192, 1024);
-    const uint64_t d_v0 = desc_sw128(smem_u32(sm + S_V), 8192, 1024);
-    const uint64_t d_v1 = desc_sw128(smem_u32(sm + S_STAGE + S_V), 8192, 1024);
-    const uint64_t d_s = desc_sw128(smem_u32(sS), 16384, 1024);
-
-    uint64_t *pending = nullptr;
-    uint32_t pending_par = 0;
-    for (int ci = 0; ci < nchunks; ++ci) {
-        const uint32_t par = (uint32_t)(ci & 1);
-        uint8_t *st = sm + par * S_STAGE;
-        const int64_t c0 = t0 + (int64_t)ci * CH;
-        const int nr = (int)(t1 - c0 < CH ? t1 - c0 : CH);
-
-        // this chunk's operands and v slice
-        const bool got = mbar_wait(&bar_ld[par], (uint32_t)(ci >> 1) & 1u, kWaitCycles);
-        asm volatile("cp.async.wait_group 0;" ::: "memory");
-        if (!got) s_abort = 1;
-        fence_async_smem();
-        tc_fence_before();
-        __syncthreads();
-        if (s_abort) { pending = &bar_ld[par]; pending_par = (uint32_t)(ci >> 1) & 1u; break; }
-        tc_fence_after();
-        if (ci + 1 < nchunks) issue_loads(ci + 1);
-
-        // state: apply the pending decay; bf16 copy for the product; store back with this
-        // chunk's decay applied now (block path) or deferred (fast path)
-        {
-            const bool fast = *reinterpret_cast<const int *>(st + SLOT_FLAG) != 0;
-            float v[32];
-            tmem_ld32(T_S + lane_off + half * 32, v);
+    if (warp == 9) {
+        // ------------------------------------------------------------------ loads
+        if (lane == 0) {
+            for (int ci = 0; ci < nchunks; ++ci) {
+                const int par = ci & 1;
+                if (ci >= 2 && !mbar_wait(&bar_free[par], (uint32_t)((ci - 2) >> 1) & 1u, kWaitCycles)) {
+                    s_abort = 1;
+                    break;
+                }
+                if (s_abort) break;
+                uint8_t *st = sm + par * S_STAGE;
+                const uint8_t *src = ws + ((size_t)(base + ci) * H + h) * SLOT_BYTES;
+                mbar_arrive_expect_tx(&bar_ld[par], SLOT_BYTES + 8192);
 #pragma unroll
-            for (int i = 0; i < 32; ++i) v[i] *= pend;
-#pragma unroll
-            for (int m = 0; m < 4; ++m) *(uint4 *)(sS + sw128_chunk(trow, 4 * half + m)) = pack8(v + 8 * m);
-            const float gdec = reinterpret_cast<const float *>(st + SLOT_GC)[trow];
-            if (!fast) {
-#pragma unroll
-                for (int i = 0; i < 32; ++i) v[i] *= gdec;
+                for (int part = 0; part < 4; ++part)
+                    bulk_g2s(st + part * (SLOT_BYTES / 4), src + part * (SLOT_BYTES / 4), SLOT_BYTES / 4,
+                             &bar_ld[par]);
+                tma_load_3d(st + S_V, &tmap_v, tile * DVT, h, (int)(t0 + (int64_t)ci * CH), &bar_ld[par]);
+                s_issued = ci + 1;
             }
-            tmem_st32(T_S + lane_off + half * 32, v);
-            pend = fast ? gdec : 1.f;
         }
-        fence_async_smem();
-        tc_fence_before();
-        __syncthreads();
-        tc_fence_after();
-
-        // [u; o] = [T'; P T'] v + [-W; Q'] S.  Descriptor start addresses advance in 16-byte
-        // units: +2 per 16 columns of a K-major line, +128 per 16 lines of an MN-major tile.
-        if (tid == 0) {
+    } else if (warp == 8) {
+        // ------------------------------------------------------------------ tensor-core issue
+        if (lane == 0) {
+            const uint64_t d_tp0 = desc_sw128(smem_u32(sm + SLOT_TP), 16, 1024);
+            const uint64_t d_a20 = desc_sw128(smem_u32(sm + SLOT_A2), 16, 1024);
+            const uint64_t d_kc0 = desc_sw128(smem_u32(sm + SLOT_KC), 8192, 1024);
+            const uint64_t d_v0 = desc_sw128(smem_u32(sm + S_V), 8192, 1024);
+            const uint64_t d_s = desc_sw128(smem_u32(sS), 16384, 1024);
+            const uint64_t d_stage = (uint64_t)(S_STAGE >> 4);      // one stage further, 16-byte units
             const uint32_t idesc = idesc_bf16(128, DVT, false, true);
-            const uint64_t dtp = par ? d_tp1 : d_tp0, dv = par ? d_v1 : d_v0, da2 = par ? d_a21 : d_a20;
+            const uint32_t idesc_s = idesc_bf16(128, DVT, true, true);
+            // Descriptor start addresses advance in 16-byte units: +2 per 16 columns of a K-major
+            // line, +128 per 16 lines of an MN-major tile.
+            for (int ci = 0; ci < nchunks; ++ci) {
+                const uint32_t par = (uint32_t)(ci & 1);
+                const uint32_t T_UO = tmem + 64 + 64 * par;
+                const uint64_t so = par ? d_stage : 0;
+                bool ok = mbar_wait(&bar_ld[par], (uint32_t)(ci >> 1) & 1u, kWaitCycles);
+                if (ok && ci >= 2) ok = mbar_wait(&bar_ofree[par], (uint32_t)((ci - 2) >> 1) & 1u, kWaitCycles);
+                if (!ok || s_abort) { s_abort = 1; break; }
+                tc_fence_after();
 #pragma unroll
-            for (int ks = 0; ks < 4; ++ks) mma_bf16(T_UO, dtp + 2 * ks, dv + 128 * ks, idesc, ks > 0);
+                for (int ks = 0; ks < 4; ++ks)
+                    mma_bf16(T_UO, d_tp0 + so + 2 * ks, d_v0 + so + 128 * ks, idesc, ks > 0);
+                if (!mbar_wait(&bar_sready, par, kWaitCycles) || s_abort) {
+                    mma_commit(&bar_uo);          // the products issued above must finish before exit
+                    s_last = 1;
+                    s_last_par = par;
+                    s_abort = 1;
+                    break;
+                }
+                tc_fence_after();
 #pragma unroll
-            for (int ks = 0; ks < 8; ++ks)
-                mma_bf16(T_UO, da2 + (ks >> 2) * 1024 + 2 * (ks & 3), d_s + 128 * ks, idesc, 1);
-            mma_commit(&bar_uo);
+                for (int ks = 0; ks < 8; ++ks)
+                    mma_bf16(T_UO, d_a20 + so + (ks >> 2) * 1024 + 2 * (ks & 3), d_s + 128 * ks, idesc, 1);
+                mma_commit(&bar_uo);
+                s_last = 1;
+                s_last_par = par;
+                if (!mbar_wait(&bar_uready, par, kWaitCycles) || s_abort) { s_abort = 1; break; }
+                tc_fence_after();
+#pragma unroll
+                for (int ks = 0; ks < 4; ++ks)
+                    mma_bf16(T_S, d_kc0 + so + 128 * ks, d_v0 + so + 128 * ks, idesc_s, 1);
+                mma_commit(&bar_s);
+                mma_commit(&bar_free[par]);
+                s_last = 2;
+                s_last_par = par;
+            }
         }
-        if (!mbar_wait(&bar_uo, par, kWaitCycles)) s_abort = 1;
-        tc_fence_after();
-        {
+    } else {
+        // ------------------------------------------------------------------ read-out
+        const bool u_warp = quarter < 2;
+        for (int ci = 0; ci < nchunks; ++ci) {
+            const uint32_t par = (uint32_t)(ci & 1);
+            uint8_t *st = sm + par * S_STAGE;
+            const uint32_t T_UO = tmem + 64 + 64 * par;
+            const int64_t c0 = t0 + (int64_t)ci * CH;
+            const int nr = (int)(t1 - c0 < CH ? t1 - c0 : CH);
+            bool ok = ci == 0 || mbar_wait(&bar_s, (uint32_t)(ci - 1) & 1u, kWaitCycles);
+            if (ok) ok = mbar_wait(&bar_ld[par], (uint32_t)(ci >> 1) & 1u, kWaitCycles);
+            if (!ok) s_abort = 1;
+            if (s_abort) break;
+            tc_fence_after();
+            // state: apply the pending decay; bf16 copy for the product; store back with this
+            // chunk's decay applied now (block path) or deferred (fast path)
+            {
+                const bool fast = *reinterpret_cast<const int *>(st + SLOT_FLAG) != 0;
+                float v[32];
+                tmem_ld32(T_S + lane_off + half * 32, v);
+#pragma unroll
+                for (int i = 0; i < 32; ++i) v[i] *= pend;
+#pragma unroll
+                for (int m = 0; m < 4; ++m) *(uint4 *)(sS + sw128_chunk(trow, 4 * half + m)) = pack8(v + 8 * m);
+                const float gdec = reinterpret_cast<const float *>(st + SLOT_GC)[trow];
+                if (!fast) {
+#pragma unroll
+                    for (int i = 0; i < 32; ++i) v[i] *= gdec;
+                }
+                tmem_st32(T_S + lane_off + half * 32, v);
+                pend = fast ? gdec : 1.f;
+            }
+            fence_async_smem();
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&bar_sready);
+            if (!mbar_wait(&bar_uo, par, kWaitCycles)) s_abort = 1;
+            if (s_abort) break;
+            tc_fence_after();
             float v[32];
             tmem_ld32(T_UO + lane_off + half * 32, v);
             uint4 pk[4];
 #pragma unroll
             for (int m = 0; m < 4; ++m) pk[m] = pack8(v + 8 * m);
-            if (trow < 64) {
+            if (u_warp) {
+                // u -> the v space of this stage (the first product has read v)
 #pragma unroll
                 for (int m = 0; m < 4; ++m) *(uint4 *)(st + S_V + sw128_chunk(trow, 4 * half + m)) = pk[m];
-            } else if (trow - 64 < nr) {
-                uint4 *dst = reinterpret_cast<uint4 *>(
-                    og + ((size_t)(c0 + trow - 64) * H + h) * DV + tile * DVT + half * 32);
+                fence_async_smem();
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&bar_uready);
+            } else {
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&bar_ofree[par]);
+                if (trow - 64 < nr) {
+                    uint4 *dst = reinterpret_cast<uint4 *>(
+                        og + ((size_t)(c0 + trow - 64) * H + h) * DV + tile * DVT + half * 32);
 #pragma unroll
-                for (int m = 0; m < 4; ++m) dst[m] = pk[m];
+                    for (int m = 0; m < 4; ++m) dst[m] = pk[m];
+                }
             }
         }
-        fence_async_smem();
-        tc_fence_before();
-        __syncthreads();
-        if (s_abort) { pending = &bar_uo; pending_par = par; break; }
-        tc_fence_after();
-
-        // S += (update operand)^T u
-        if (tid == 0) {
-            const uint64_t dkc = par ? d_kc1 : d_kc0, du = par ? d_v1 : d_v0;
-#pragma unroll
-            for (int ks = 0; ks < 4; ++ks)
-                mma_bf16(T_S, dkc + 128 * ks, du + 128 * ks, idesc_bf16(128, DVT, true, true), 1);
-            mma_commit(&bar_s);
-        }
-        if (!mbar_wait(&bar_s, par, kWaitCycles)) s_abort = 1;
-        tc_fence_after();
-        __syncthreads();
-        if (s_abort) { pending = &bar_s; pending_par = par; break; }
     }
-    asm volatile("cp.async.wait_all;" ::: "memory");
+    __syncthreads();
 
-    if (pending) {
-        // A wait gave up: record it, give the in-flight work one more bounded wait, and
+    bool failed = s_abort != 0;
+    if (!failed && nchunks > 0) {
+        if (s_last != 2 || !mbar_wait(&bar_s, (uint32_t)(nchunks - 1) & 1u, kWaitCycles)) failed = true;
+    }
+    if (failed) {
+        // A wait gave up: record it, give the last committed product and every load still in
+        // flight one more bounded wait (shared memory must not be released under them), and
         // leave without writing the state.
         if (tid == 0) atomicOr(&g_kda_device_status, 1u);
-        mbar_wait(pending, pending_par, kWaitCycles);
-    } else if (a.S_final) {
+        if (s_last == 1) mbar_wait(&bar_uo, s_last_par, kWaitCycles);
+        if (s_last == 2) mbar_wait(&bar_s, s_last_par, kWaitCycles);
+        for (int ci = s_issued - 2 > 0 ? s_issued - 2 : 0; ci < s_issued; ++ci)
+            mbar_wait(&bar_ld[ci & 1], (uint32_t)(ci >> 1) & 1u, kWaitCycles);
+    } else if (a.S_final && tid < kReadoutThreads) {
+        tc_fence_after();
         float v[32];
         tmem_ld32(T_S + lane_off + half * 32, v);
         float4 *dst = reinterpret_cast<float4 *>(a.S_final + s_base + (size_t)trow * DV);
@@ -815,7 +876,7 @@ __global__ void __launch_bounds__(NTHR, 1)
     }
     tc_fence_before();
     __syncthreads();
-    if (warp == 0) tmem_free(tmem, 128);
+    if (warp == 0) tmem_free(tmem, 256);
 }
 
 bool g_configured[64] = {};
@@ -847,6 +908,34 @@ cudaError_t configure_pool(int dev) {
     return cudaSuccess;
 }
 
+// Tensor map of v viewed as [T_total][H][d_v] bf16: boxes of 64 d_v columns x 1 head x 64
+// tokens, 128-byte swizzle, so one TMA load gives the scan its v tile in the MMA layout.
+// Tokens past T_total read as zeros; tokens of the next sequence that fill a partial last
+// chunk only meet zero columns of [T'; P T'].
+PFN_cuTensorMapEncodeTiled_v12000 g_encode_tiled = nullptr;
+
+cudaError_t encode_v_map(const KdaChunkArgs &a, CUtensorMap *map) {
+    memset(map, 0, sizeof(*map));
+    if (a.T_total == 0) return cudaSuccess;       // no chunk: the map is never read
+    if (g_encode_tiled == nullptr) {
+        void *fn = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        const cudaError_t e = cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q);
+        if (e != cudaSuccess) return e;
+        if (q != cudaDriverEntryPointSuccess || fn == nullptr) return cudaErrorNotSupported;
+        g_encode_tiled = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
+    }
+    const cuuint64_t dims[3] = {(cuuint64_t)DV, (cuuint64_t)a.H, (cuuint64_t)a.T_total};
+    const cuuint64_t strides[2] = {(cuuint64_t)DV * 2, (cuuint64_t)a.H * DV * 2};
+    const cuuint32_t box[3] = {(cuuint32_t)DVT, 1, (cuuint32_t)CH};
+    const cuuint32_t estr[3] = {1, 1, 1};
+    const CUresult r = g_encode_tiled(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(a.v), dims,
+                                      strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                                      CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                                      CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
+}
+
 int64_t max_slots_of(const KdaChunkArgs &a) {
     return a.cu_seqlens ? (a.T_total + CH - 1) / CH + a.N : (int64_t)a.N * ((a.T + CH - 1) / CH);
 }
@@ -875,8 +964,10 @@ cudaError_t kda_launch_chunk_tc_ws(const KdaChunkArgs &a, void *ws, cudaStream_t
         const dim3 grid((unsigned)max_slots, (unsigned)a.H);
         kda_chunk_intra_kernel<<<grid, NTHR, kIntraSmem, stream>>>(a, slots, slot_base);
     }
-    kda_chunk_scan_kernel<<<(unsigned)((int64_t)a.N * a.H * NTILE), NTHR, kScanSmem, stream>>>(a, slots,
-                                                                                             slot_base);
+    CUtensorMap tmap_v;
+    if ((e = encode_v_map(a, &tmap_v)) != cudaSuccess) return e;
+    kda_chunk_scan_kernel<<<(unsigned)((int64_t)a.N * a.H * NTILE), SCAN_THREADS, kScanSmem, stream>>>(
+        a, slots, slot_base, tmap_v);
     return cudaGetLastError();
 }
 
