@@ -457,30 +457,57 @@ __global__ void __launch_bounds__(NTHR, 2)
     }
     __syncthreads();
 
-    // ---------------- T = (I + A)^{-1}: diagonal 16 x 16 blocks.  Warp w < 4 solves block w:
-    //      lane i and lane i + 16 both carry column i; each sums half of every row's terms
-    //      (even / odd m) and one shuffle joins them.
+    // ---------------- T = (I + A)^{-1}: diagonal 16 x 16 blocks.  Warp w < 4 solves block w by
+    //      forward substitution: lane i holds row i of the block of A and column i of T; row r
+    //      of A is broadcast from lane r.
+    //      Meanwhile warps 4-7 write the identity half of [I; P] and preload the accumulator of
+    //      the W product with [0; s q gamma], so that it yields [-W; s q gamma - P W] directly.
     if (warp < 4) {
-        const int w = warp, i = lane & 15, odd = lane >> 4;
+        const int w = warp, i = lane & 15;
         const float *Ab = Am + (16 * w) * LF + 16 * w;
-        float tc[16];
+        float arow[16];
+#pragma unroll
+        for (int m = 0; m < 16; ++m) arow[m] = Ab[i * LF + m];
+        float tcol[16];
 #pragma unroll
         for (int r = 0; r < 16; ++r) {
-            float acc0 = 0.f, acc1 = 0.f;
+            float acc = 0.f;
 #pragma unroll
-            for (int m = 0; m < r; ++m) {
-                if ((m & 1) == odd && m >= i) {
-                    if (m & 2) acc1 = fmaf(Ab[r * LF + m], tc[m], acc1);
-                    else acc0 = fmaf(Ab[r * LF + m], tc[m], acc0);
+            for (int m = 0; m < r; ++m) acc = fmaf(__shfl_sync(0xffffffffu, arow[m], r), tcol[m], acc);
+            tcol[r] = r < i ? 0.f : (r == i ? 1.f : -acc);
+        }
+        if (lane < 16) {
+#pragma unroll
+            for (int r = 0; r < 16; ++r) Tm[(16 * w + r) * LF + 16 * w + i] = tcol[r];
+        }
+    } else {
+        for (int o = tid - 128; o < 512; o += 128) {       // lines 0-63 of [I; P]: the identity
+            const int l = o >> 3, j = o & 7;
+            float v8[8];
+#pragma unroll
+            for (int e = 0; e < 8; ++e) v8[e] = 8 * j + e == l ? 1.f : 0.f;
+            *(uint4 *)(sIP + sw128_chunk(l, j)) = pack8(v8);
+        }
+#pragma unroll
+        for (int part = 0; part < 4; ++part) {             // 32 columns of the W accumulator each
+            float v[32];
+            if (trow < 64) {
+#pragma unroll
+                for (int e = 0; e < 32; ++e) v[e] = 0.f;
+            } else {
+#pragma unroll
+                for (int m = 0; m < 4; ++m) {              // s q gamma of row trow - 64 (KQ tile)
+                    const uint4 pk = *(const uint4 *)(sKQ + (part >> 1) * 16384 + sw128_chunk(trow, 4 * (part & 1) + m));
+                    const uint32_t w4[4] = {pk.x, pk.y, pk.z, pk.w};
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        const float2 qq = unpack_bf16(w4[e]);
+                        v[8 * m + 2 * e] = qq.x;
+                        v[8 * m + 2 * e + 1] = qq.y;
+                    }
                 }
             }
-            const float part = acc0 + acc1;
-            const float tot = part + __shfl_xor_sync(0xffffffffu, part, 16);
-            tc[r] = r < i ? 0.f : (r == i ? 1.f : -tot);
-        }
-        if (!odd) {
-#pragma unroll
-            for (int r = 0; r < 16; ++r) Tm[(16 * w + r) * LF + 16 * w + i] = tc[r];
+            tmem_st32(T_W + lane_off + 32 * part, v);
         }
     }
     __syncthreads();
@@ -527,11 +554,11 @@ __global__ void __launch_bounds__(NTHR, 2)
             __syncthreads();
         }
     }
-    //      T' (lines 0-63 of [T'; P T']) and the identity half of [I; P], 8 elements at a time
-    for (int o = tid; o < 1024; o += NTHR) {
+    //      T' (lines 0-63 of [T'; P T']), 8 elements at a time
+    for (int o = tid; o < 512; o += NTHR) {
         const int l = o >> 3, j = o & 7;
         float v8[8];
-        if (l < 64) {
+        {
             const float4 t0v = *reinterpret_cast<const float4 *>(&Tm[l * LF + 8 * j]);
             const float4 t1v = *reinterpret_cast<const float4 *>(&Tm[l * LF + 8 * j + 4]);
             const float4 b0 = *reinterpret_cast<const float4 *>(&sBeta[8 * j]);
@@ -541,11 +568,6 @@ __global__ void __launch_bounds__(NTHR, 2)
 #pragma unroll
             for (int e = 0; e < 8; ++e) v8[e] = 8 * j + e <= l ? tv[e] : 0.f;
             *(uint4 *)(sTP + sw128_chunk(l, j)) = pack8(v8);
-        } else {
-            const int pl = l - 64;
-#pragma unroll
-            for (int e = 0; e < 8; ++e) v8[e] = 8 * j + e == pl ? 1.f : 0.f;
-            *(uint4 *)(sIP + sw128_chunk(pl, j)) = pack8(v8);
         }
     }
     fence_async_smem();
@@ -575,13 +597,14 @@ __global__ void __launch_bounds__(NTHR, 2)
     __syncthreads();
     tc_fence_after();
 
-    // ---------------- [W; P W] = [T'; P T'] (k gamma); meanwhile [T'; P T'] goes to the slot
+    // ---------------- [-W; s q gamma - P W] = [0; s q gamma] - [T'; P T'] (k gamma); meanwhile
+    //      [T'; P T'] goes to the slot
     if (tid == 0) {
         const uint32_t a0 = smem_u32(sTP), b0 = smem_u32(sKQ);
 #pragma unroll
         for (int ks = 0; ks < 4; ++ks)
             mma_bf16(T_W, desc_sw128(a0 + 32 * ks, 16, 1024), desc_sw128(b0 + 2048 * ks, 16384, 1024),
-                     idesc_bf16(128, 128, false, true), ks > 0);
+                     idesc_bf16(128, 128, false, true, true), 1);
         mma_commit(&bar_w);
     }
     if (tid == 32) {
@@ -597,22 +620,6 @@ __global__ void __launch_bounds__(NTHR, 2)
     for (int part = 0; part < 2; ++part) {
         float v[32];
         tmem_ld32(T_W + lane_off + half * 64 + part * 32, v);
-        if (trow >= 64) {
-#pragma unroll
-            for (int m = 0; m < 4; ++m) {    // s q gamma of row trow - 64, from the KQ tile
-                const uint4 pk = *(const uint4 *)(sKQ + half * 16384 + sw128_chunk(trow, 4 * part + m));
-                const uint32_t w4[4] = {pk.x, pk.y, pk.z, pk.w};
-#pragma unroll
-                for (int e = 0; e < 4; ++e) {
-                    const float2 qq = unpack_bf16(w4[e]);
-                    v[8 * m + 2 * e] = qq.x - v[8 * m + 2 * e];
-                    v[8 * m + 2 * e + 1] = qq.y - v[8 * m + 2 * e + 1];
-                }
-            }
-        } else {
-#pragma unroll
-            for (int i = 0; i < 32; ++i) v[i] = -v[i];
-        }
 #pragma unroll
         for (int m = 0; m < 4; ++m)
             *(uint4 *)(sA2 + half * 16384 + sw128_chunk(trow, 4 * part + m)) = pack8(v + 8 * m);
