@@ -87,13 +87,15 @@ static_assert(I_CP + 4096 <= I_TP, "block-path scratch inside T");
 static_assert(I_AM + 32768 <= I_TP, "[-W; s q gamma - P W] staged in the space of A and T");
 static_assert(2 * (kIntraSmem + 1024) <= 233472, "two intra CTAs per SM");
 
-// Scan kernel shared memory: two stages of {slot image, v slice}, the bf16 state copy.
+// Scan kernel shared memory: two stages of {slot image, v slice}, the bf16 state copy, two o
+// staging tiles.
 constexpr uint32_t S_STAGE = 74752;     // SLOT_BYTES + 8192 (v slice), 1024-aligned
 constexpr uint32_t S_V = SLOT_BYTES;    // v slice of the chunk, then u: 64 lines (MN-major B)
 constexpr uint32_t S_S = 2 * S_STAGE;   // bf16 state copy: 128 lines (MN-major B)
-constexpr uint32_t S_END = S_S + 16384;
+constexpr uint32_t S_O = S_S + 16384;   // o of a chunk's d_v tile, [64 tokens][64] bf16 (one TMA box)
+constexpr uint32_t S_END = S_O + 2 * 8192;
 constexpr size_t kScanSmem = S_END + 1024;
-static_assert(S_STAGE % 1024 == 0 && S_V % 1024 == 0 && S_S % 1024 == 0, "tile alignment");
+static_assert(S_STAGE % 1024 == 0 && S_V % 1024 == 0 && S_S % 1024 == 0 && S_O % 1024 == 0, "tile alignment");
 static_assert(kScanSmem <= 232448, "shared memory budget");
 
 __constant__ int kPairA[10] = {0, 1, 1, 2, 2, 2, 3, 3, 3, 3};
@@ -647,18 +649,22 @@ __global__ void __launch_bounds__(NTHR, 2)
 //   warp 8     tensor-core issue (one thread): [u; o] = [T'; P T'] v as soon as the chunk is in
 //              shared memory, + [-W; s q gamma - P W] S once S is copied, S += KC^T u once u is;
 //   warp 9     loads (one thread): slot c and the v tile of chunk c into stage c & 1 once the
-//              state product of chunk c - 2 has released it.
+//              state product of chunk c - 2 has released it;
+//   warp 10    stores (one thread): o of a full chunk, staged in shared memory by the o warps,
+//              to HBM by one TMA store (a partial last chunk is stored directly by the o warps,
+//              so no box reaches into the next sequence's tokens).
 // [u; o] alternates between two TMEM accumulators so chunk c + 1's first product can start
 // while o of chunk c is still being read.
-constexpr int SCAN_THREADS = 320;
+constexpr int SCAN_THREADS = 352;
 constexpr int kReadoutThreads = 256;
 
 __global__ void __launch_bounds__(SCAN_THREADS, 1)
     kda_chunk_scan_kernel(KdaChunkArgs a, const uint8_t *ws, const int32_t *slot_base,
-                          const __grid_constant__ CUtensorMap tmap_v) {
+                          const __grid_constant__ CUtensorMap tmap_v, const __grid_constant__ CUtensorMap tmap_o) {
     extern __shared__ uint8_t smraw[];
     uint8_t *sm = smraw + ((1024u - (smem_u32(smraw) & 1023u)) & 1023u);   // stays a shared-space pointer
     __shared__ uint64_t bar_ld[2], bar_free[2], bar_ofree[2], bar_sready, bar_uo, bar_uready, bar_s;
+    __shared__ uint64_t bar_ostaged[2], bar_obuf[2];
     __shared__ uint32_t s_tmem;
     __shared__ volatile int s_abort;
     __shared__ int s_last, s_issued;      // last commit of the issuing thread (0 none, 1 uo, 2 s); loads issued
@@ -680,6 +686,8 @@ __global__ void __launch_bounds__(SCAN_THREADS, 1)
             mbar_init(&bar_ld[i], 1);
             mbar_init(&bar_free[i], 1);
             mbar_init(&bar_ofree[i], 4);
+            mbar_init(&bar_ostaged[i], 4);
+            mbar_init(&bar_obuf[i], 1);
         }
         mbar_init(&bar_sready, 8);
         mbar_init(&bar_uo, 1);
@@ -742,6 +750,25 @@ __global__ void __launch_bounds__(SCAN_THREADS, 1)
                 tma_load_3d(st + S_V, &tmap_v, tile * DVT, h, (int)(t0 + (int64_t)ci * CH), &bar_ld[par]);
                 s_issued = ci + 1;
             }
+        }
+    } else if (warp == 10) {
+        // ------------------------------------------------------------------ o stores
+        if (lane == 0) {
+            for (int ci = 0; ci < nchunks; ++ci) {
+                const uint32_t b = (uint32_t)(ci & 1);
+                if (!mbar_wait(&bar_ostaged[b], (uint32_t)(ci >> 1) & 1u, kWaitCycles) || s_abort) {
+                    s_abort = 1;
+                    break;
+                }
+                const int64_t c0 = t0 + (int64_t)ci * CH;
+                if (t1 - c0 >= CH) {
+                    tma_store_3d(&tmap_o, sm + S_O + b * 8192, tile * DVT, h, (int)c0);
+                    bulk_commit();
+                }
+                bulk_wait_read_all();
+                mbar_arrive(&bar_obuf[b]);
+            }
+            bulk_wait_read_all();
         }
     } else if (warp == 8) {
         // ------------------------------------------------------------------ tensor-core issue
@@ -848,12 +875,23 @@ __global__ void __launch_bounds__(SCAN_THREADS, 1)
                 tc_fence_before();
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&bar_ofree[par]);
-                if (trow - 64 < nr) {
+                // o into the staging tile of this chunk parity (free once the TMA store of chunk
+                // ci - 2 has read it), or straight to HBM for a partial chunk
+                if (nr == CH) {
+                    if (ci >= 2 && !mbar_wait(&bar_obuf[par], (uint32_t)((ci - 2) >> 1) & 1u, kWaitCycles))
+                        s_abort = 1;
+                    uint8_t *so = sm + S_O + par * 8192;
+#pragma unroll
+                    for (int m = 0; m < 4; ++m) *(uint4 *)(so + sw128_chunk(trow - 64, 4 * half + m)) = pk[m];
+                    fence_async_smem();
+                } else if (trow - 64 < nr) {
                     uint4 *dst = reinterpret_cast<uint4 *>(
                         og + ((size_t)(c0 + trow - 64) * H + h) * DV + tile * DVT + half * 32);
 #pragma unroll
                     for (int m = 0; m < 4; ++m) dst[m] = pk[m];
                 }
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&bar_ostaged[par]);
             }
         }
     }
@@ -915,13 +953,14 @@ cudaError_t configure_pool(int dev) {
     return cudaSuccess;
 }
 
-// Tensor map of v viewed as [T_total][H][d_v] bf16: boxes of 64 d_v columns x 1 head x 64
-// tokens, 128-byte swizzle, so one TMA load gives the scan its v tile in the MMA layout.
-// Tokens past T_total read as zeros; tokens of the next sequence that fill a partial last
-// chunk only meet zero columns of [T'; P T'].
+// Tensor map of v or o viewed as [T_total][H][d_v] bf16: boxes of 64 d_v columns x 1 head x
+// 64 tokens, 128-byte swizzle, so one TMA load gives the scan its v tile in the MMA layout and
+// one TMA store writes a chunk's o tile.  Tokens past T_total read as zeros; tokens of the next
+// sequence that fill a partial last chunk of v only meet zero columns of [T'; P T'], and o of a
+// partial chunk is never stored by TMA.
 PFN_cuTensorMapEncodeTiled_v12000 g_encode_tiled = nullptr;
 
-cudaError_t encode_v_map(const KdaChunkArgs &a, CUtensorMap *map) {
+cudaError_t encode_tok_map(const KdaChunkArgs &a, const void *base, CUtensorMap *map) {
     memset(map, 0, sizeof(*map));
     if (a.T_total == 0) return cudaSuccess;       // no chunk: the map is never read
     if (g_encode_tiled == nullptr) {
@@ -936,7 +975,7 @@ cudaError_t encode_v_map(const KdaChunkArgs &a, CUtensorMap *map) {
     const cuuint64_t strides[2] = {(cuuint64_t)DV * 2, (cuuint64_t)a.H * DV * 2};
     const cuuint32_t box[3] = {(cuuint32_t)DVT, 1, (cuuint32_t)CH};
     const cuuint32_t estr[3] = {1, 1, 1};
-    const CUresult r = g_encode_tiled(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(a.v), dims,
+    const CUresult r = g_encode_tiled(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(base), dims,
                                       strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
                                       CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                                       CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
@@ -971,10 +1010,11 @@ cudaError_t kda_launch_chunk_tc_ws(const KdaChunkArgs &a, void *ws, cudaStream_t
         const dim3 grid((unsigned)max_slots, (unsigned)a.H);
         kda_chunk_intra_kernel<<<grid, NTHR, kIntraSmem, stream>>>(a, slots, slot_base);
     }
-    CUtensorMap tmap_v;
-    if ((e = encode_v_map(a, &tmap_v)) != cudaSuccess) return e;
+    CUtensorMap tmap_v, tmap_o;
+    if ((e = encode_tok_map(a, a.v, &tmap_v)) != cudaSuccess) return e;
+    if ((e = encode_tok_map(a, a.out, &tmap_o)) != cudaSuccess) return e;
     kda_chunk_scan_kernel<<<(unsigned)((int64_t)a.N * a.H * NTILE), SCAN_THREADS, kScanSmem, stream>>>(
-        a, slots, slot_base, tmap_v);
+        a, slots, slot_base, tmap_v, tmap_o);
     return cudaGetLastError();
 }
 

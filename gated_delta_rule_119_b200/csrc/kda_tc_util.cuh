@@ -119,6 +119,15 @@ __device__ __forceinline__ void tma_load_3d(void *dst_smem, const void *tmap, in
         : "memory");
 }
 
+// Tiled TMA store of one box of a 3-D tensor map from this CTA's shared memory, tracked in
+// this thread's bulk async-group.  Coordinates must not be negative.
+__device__ __forceinline__ void tma_store_3d(const void *tmap, const void *src_smem, int x, int y, int z) {
+    asm volatile("cp.async.bulk.tensor.3d.global.shared::cta.tile.bulk_group [%0, {%2, %3, %4}], [%1];" ::"l"(
+                     reinterpret_cast<uint64_t>(tmap)),
+                 "r"(smem_u32(src_smem)), "r"(x), "r"(y), "r"(z)
+                 : "memory");
+}
+
 // Bulk asynchronous global -> shared copy (16-byte aligned addresses, size a multiple of 16);
 // completion is counted on `bar` in bytes.
 __device__ __forceinline__ void bulk_g2s(void *dst_smem, const void *src, uint32_t bytes, uint64_t *bar) {
