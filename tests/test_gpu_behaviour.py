@@ -1,0 +1,91 @@
+"""GPU behaviour of the C ABI beyond single-call parity: calls on a side stream, run-to-run
+determinism of the tensor-core prefill, many heads with short sequences, one sequence split
+into several calls (S_final fed back as S0).  All through libkda.so; oracle values where a
+value is checked (max|x - r| / max|r| within the dtype's bar)."""
+import numpy as np
+import pytest
+
+import oracle
+from gated_delta_rule_119_b200.inputs import make_inputs, to_torch
+
+torch = pytest.importorskip("torch")
+pytestmark = pytest.mark.gpu
+TOL = {"f32": 1e-4, "bf16": 2e-2}
+
+
+def rel_err(x, r):
+    return float(np.abs(x - r).max() / max(np.abs(r).max(), 1e-30))
+
+
+def call(d, **kw):
+    from gated_delta_rule_119_b200 import kda_chunk_fwd
+    return kda_chunk_fwd(d["q"], d["k"], d["v"], d["log_alpha"], d["beta"], d["S0"],
+                         d["cu_seqlens"], **kw)
+
+
+def test_side_stream_gives_the_default_stream_result():
+    inp = make_inputs(2, 700, 4, 128, 128, "bf16", 1201, state=True)
+    d = to_torch(inp)
+    o_ref, s_ref = call(d)
+    torch.cuda.synchronize()
+    side = torch.cuda.Stream()
+    side.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(side):
+        o, s = call(d)
+    side.synchronize()
+    assert torch.equal(o, o_ref) and torch.equal(s, s_ref)
+    from gated_delta_rule_119_b200 import kda_device_status
+    assert kda_device_status() == 0
+
+
+@pytest.mark.parametrize("gates", ["default", "extremes"])
+def test_tensor_core_path_is_deterministic(gates):
+    inp = make_inputs(2, 1000, 4, 128, 128, "bf16", 1202, state=True, gates=gates)
+    d = to_torch(inp)
+    outs = [call(d) for _ in range(3)]
+    torch.cuda.synchronize()
+    for o, s in outs[1:]:
+        assert torch.equal(o, outs[0][0]) and torch.equal(s, outs[0][1])
+
+
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+def test_many_heads_short_sequences(dtype):
+    inp = make_inputs(3, 70, 64, 128, 128, dtype, 1203, state=True)
+    d = to_torch(inp)
+    o, s = call(d)
+    torch.cuda.synchronize()
+    ro, rs = oracle.recurrent_full(inp.q, inp.k, inp.v, inp.log_alpha, inp.beta, inp.S0, inp.offsets())
+    o = o.float().cpu().numpy().reshape(inp.total_tokens, inp.H, inp.dv)
+    eo, es = rel_err(o, ro), rel_err(s.cpu().numpy(), rs)
+    print(f"[behaviour] many heads {dtype}: o {eo:.3e}  S_final {es:.3e}")
+    assert eo <= TOL[dtype] and es <= TOL[dtype]
+
+
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+def test_sequence_split_across_calls(dtype):
+    """Prefill of tokens [0, 300) then [300, 700) with the first call's S_final as the
+    second's S0 equals one call over [0, 700) (both checked against the oracle)."""
+    full = make_inputs(1, 700, 3, 128, 128, dtype, 1204, state=True)
+    cut = 300
+
+    def part(lo, hi, S0):
+        p = make_inputs(1, hi - lo, 3, 128, 128, dtype, 1204)
+        for name in ("q", "k", "v", "log_alpha", "beta"):
+            setattr(p, name, np.ascontiguousarray(getattr(full, name)[lo:hi]))
+        p.S0 = S0
+        return p
+
+    first = part(0, cut, full.S0)
+    d1 = to_torch(first)
+    o1, s1 = call(d1)
+    second = part(cut, 700, s1.cpu().numpy())
+    d2 = to_torch(second)
+    o2, s2 = call(d2)
+    torch.cuda.synchronize()
+    ro, rs = oracle.recurrent_full(full.q, full.k, full.v, full.log_alpha, full.beta, full.S0,
+                                   full.offsets())
+    o = np.concatenate([o1.float().cpu().numpy().reshape(cut, 3, 128),
+                        o2.float().cpu().numpy().reshape(700 - cut, 3, 128)])
+    eo, es = rel_err(o, ro), rel_err(s2.cpu().numpy(), rs)
+    print(f"[behaviour] split {dtype}: o {eo:.3e}  S_final {es:.3e}")
+    assert eo <= TOL[dtype] and es <= TOL[dtype]
