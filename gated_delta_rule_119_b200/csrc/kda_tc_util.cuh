@@ -108,7 +108,7 @@ __device__ __forceinline__ void mbar_arrive(uint64_t *bar) {
 }
 
 // Tiled TMA load of one box of a 3-D tensor map into this CTA's shared memory, completion
-// counted on `bar` in bytes.  No multicast.  The innermost coordinate times the element size
+// counted on `bar` in bytes; the destination is this CTA only.  The innermost coordinate times the element size
 // must be a multiple of 16 bytes.
 __device__ __forceinline__ void tma_load_3d(void *dst_smem, const void *tmap, int x, int y, int z,
                                             uint64_t *bar) {
