@@ -39,7 +39,7 @@ struct SimtLayout {
     static constexpr int LKV = LK > LV ? LK : LV;
     static constexpr size_t floats =
         (size_t)kChunk * LKV + 3 * (size_t)kChunk * LK + (size_t)kChunk * LV +
-        2 * (size_t)kChunk * LC + kChunk + DK;
+        3 * (size_t)kChunk * LC + kChunk + DK;
     static constexpr size_t bytes = floats * sizeof(float);
     static_assert(kSimtThreads % DV == 0 && DK % NSL == 0 && kChunk % NSL == 0, "tiling");
 };
@@ -57,7 +57,8 @@ __global__ void __launch_bounds__(kSimtThreads, 1) kda_chunk_simt_kernel(KdaChun
     float *Vb = Kc + CH * LK;        // [CH][LV]   v, then u
     float *Ab = Vb + CH * LV;        // [CH][LC]   A, then T'
     float *Pb = Ab + CH * LC;        // [CH][LC]   P
-    float *bt = Pb + CH * LC;        // [CH]       beta
+    float *Tb = Pb + CH * LC;        // [CH][LC]   T (lower); partial products in the upper blocks
+    float *bt = Tb + CH * LC;        // [CH]       beta
     float *dC = bt + CH;             // [DK]       e^{g_last}
 
     const int H = a.H;
@@ -164,24 +165,57 @@ __global__ void __launch_bounds__(kSimtThreads, 1) kda_chunk_simt_kernel(KdaChun
         }
         __syncthreads();
 
-        // 5. T = (I + A)^{-1}: row r of T below the diagonal is
-        //    T[r][i] = -A[r][i] - sum_{i<m<r} A[r][m] T[m][i]; rows m < r are final.
-        for (int r = 1; r < CH; ++r) {
-            float val = 0.f;
-            if (tid < r) {
-                float acc = Ab[r * LC + tid];
-                for (int m = tid + 1; m < r; ++m) acc = fmaf(Ab[r * LC + m], Ab[m * LC + tid], acc);
-                val = -acc;
+        // 5. T = (I + A)^{-1}, blocked: the four 16 x 16 diagonal blocks by forward
+        //    substitution (warp w < 4 solves block w; lane i holds row i of the block of A and
+        //    column i of T, row r of A is broadcast from lane r), then the blocks below by
+        //    distance d = a - b: T_ab = -T_aa X_ab with X_ab = sum_{m=b}^{a-1} A_am T_mb, X_ab
+        //    parked in the (unused) upper block (b, a) of Tb.
+        {
+            const int warp = tid >> 5, lane = tid & 31;
+            if (warp < 4) {
+                const int w = warp, i = lane & 15;
+                const float *Abk = Ab + (16 * w) * LC + 16 * w;
+                float arow[16], tcol[16];
+#pragma unroll
+                for (int m = 0; m < 16; ++m) arow[m] = Abk[i * LC + m];
+#pragma unroll
+                for (int r = 0; r < 16; ++r) {
+                    float acc = 0.f;
+#pragma unroll
+                    for (int m = 0; m < r; ++m) acc = fmaf(__shfl_sync(0xffffffffu, arow[m], r), tcol[m], acc);
+                    tcol[r] = r < i ? 0.f : (r == i ? 1.f : -acc);
+                }
+                if (lane < 16) {
+#pragma unroll
+                    for (int r = 0; r < 16; ++r) Tb[(16 * w + r) * LC + 16 * w + i] = tcol[r];
+                }
             }
             __syncthreads();
-            if (tid < r) Ab[r * LC + tid] = val;
-            __syncthreads();
+            for (int d = 1; d < 4; ++d) {
+                const int nb = 4 - d;                       // blocks (b + d, b), b < nb
+                for (int e = tid; e < nb * 256; e += kSimtThreads) {
+                    const int b = e >> 8, r = (e >> 4) & 15, c = e & 15, ab = b + d;
+                    float acc = 0.f;
+                    for (int m = 16 * b; m < 16 * ab; ++m)
+                        acc = fmaf(Ab[(16 * ab + r) * LC + m], Tb[m * LC + 16 * b + c], acc);
+                    Tb[(16 * b + r) * LC + 16 * ab + c] = acc;      // X_ab, row r, column c
+                }
+                __syncthreads();
+                for (int e = tid; e < nb * 256; e += kSimtThreads) {
+                    const int b = e >> 8, r = (e >> 4) & 15, c = e & 15, ab = b + d;
+                    float acc = 0.f;
+#pragma unroll
+                    for (int k = 0; k < 16; ++k)
+                        acc = fmaf(Tb[(16 * ab + r) * LC + 16 * ab + k], Tb[(16 * b + k) * LC + 16 * ab + c], acc);
+                    Tb[(16 * ab + r) * LC + 16 * b + c] = -acc;
+                }
+                __syncthreads();
+            }
         }
-        //    T' = T Diag(beta) (unit diagonal of T included).
+        //    T' = T Diag(beta) (lower triangle of T, unit diagonal included).
         for (int p = tid; p < CH * CH; p += kSimtThreads) {
             const int r = p / CH, i = p % CH;
-            const float t = i < r ? Ab[r * LC + i] : (i == r ? 1.f : 0.f);
-            Ab[r * LC + i] = t * bt[i];
+            Ab[r * LC + i] = i <= r ? Tb[r * LC + i] * bt[i] : 0.f;
         }
         __syncthreads();
 
