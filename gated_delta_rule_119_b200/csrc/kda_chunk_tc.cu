@@ -63,18 +63,16 @@ constexpr uint32_t SLOT_KC = 49152;     // update operand: 2 x 64 lines (MN-majo
 constexpr uint32_t SLOT_GC = 65536;     // gamma_last [128] fp32
 constexpr uint32_t SLOT_FLAG = 66048;   // 1 = fast path (decay deferred), 0 = block path
 constexpr uint32_t SLOT_BYTES = 66560;
-// The block path parks its factored operands in the slot before it is filled (row-major
-// [64][128] bf16): left k, right k, left s q.
-constexpr uint32_t SLOT_KL = 0, SLOT_KR = 16384, SLOT_QL = 32768;
 
 // Intra-chunk kernel shared memory (bytes from a 1024-aligned base); two CTAs per SM.
 constexpr uint32_t I_KQ = 0;            // [k gamma; s q gamma]: 2 x 128 lines
-constexpr uint32_t I_KC = 32768;        // k e^-g (fast-path B operand of A, P), then [I; P]
-constexpr uint32_t I_AM = 49152;        // A [64][LF] fp32
+constexpr uint32_t I_KC = 32768;        // k e^-g (fast-path B operand of A, P) or the block
+                                        //   path's right k factor, then [I; P]
+constexpr uint32_t I_AM = 49152;        // the block path's left k factor, then A [64][LF] fp32
 constexpr uint32_t I_TM = 66560;        // T [64][LF] fp32; before it, the block path's scale
                                         //   table [10][128] and exact-path P [4][16][16]
-constexpr uint32_t I_SC = I_TM, I_CP = I_TM + 5120;
-constexpr uint32_t I_TP = 83968;        // [T'; P T']: 128 lines
+constexpr uint32_t I_SC = I_TM, I_CP = I_TM + 5120, I_CA = I_TM + 9216;   // I_CA: exact-path A [4][16][16]
+constexpr uint32_t I_TP = 83968;        // q (then the block path's left s q factor), then [T'; P T']
 constexpr uint32_t I_BETA = 100352;     // [64]
 constexpr uint32_t I_GC = I_BETA + 256; // [128]
 constexpr uint32_t I_BS = I_GC + 512;   // [4][128] sum of log_alpha per 16-row block
@@ -83,7 +81,7 @@ constexpr uint32_t I_XT = I_BT + 2048;  // [6][128] forward-substitution scratch
 constexpr uint32_t I_END = I_XT + 3072;
 constexpr size_t kIntraSmem = I_END + 1024;
 static_assert(I_TP % 1024 == 0 && I_KC % 1024 == 0, "tile alignment");
-static_assert(I_CP + 4096 <= I_TP, "block-path scratch inside T");
+static_assert(I_CA + 4096 <= I_TP, "block-path scratch inside T");
 static_assert(I_AM + 32768 <= I_TP, "[-W; s q gamma - P W] staged in the space of A and T");
 static_assert(2 * (kIntraSmem + 1024) <= 233472, "two intra CTAs per SM");
 
@@ -110,6 +108,13 @@ __device__ __forceinline__ uint4 pack8(const float *v) {
     return pk;
 }
 
+// Byte offset of element (r, c) of a [64][128] bf16 row-major tile whose 16-byte chunks are
+// XOR-swizzled by r & 7: conflict-free both for a warp reading 32 consecutive channels of one
+// row and for the warp-MMA fragment loads (8 rows x 4 column pairs).
+__device__ __forceinline__ uint32_t rm_sw(int r, int c) {
+    return (uint32_t)(r * 256 + (((c >> 3) ^ (r & 7)) << 4) + ((c & 7) << 1));
+}
+
 // Slot bases of the sequences: base[n] = sum_{m<n} ceil(len_m / 64).
 __global__ void kda_chunk_slots_kernel(const int32_t *cu_seqlens, int N, int64_t T_total, int32_t *base) {
     if (threadIdx.x != 0) return;
@@ -127,7 +132,7 @@ __global__ void kda_chunk_slots_kernel(const int32_t *cu_seqlens, int N, int64_t
 // strong for the rescaled factors: running products of alpha, inputs re-read from memory.
 // Adds beta_r k_r k_i D_ri to A (i < r) and s q_r k_i D_ri to the block's exact P sums.
 __device__ __noinline__ void exact_diag_channel(const KdaChunkArgs &a, int64_t c0, int nr, int h, int blk,
-                                                int ch, const float *sBeta, float *Am, float *sCP) {
+                                                int ch, const float *sBeta, float *sCA, float *sCP) {
     const int H = a.H;
     const __nv_bfloat16 *qg = static_cast<const __nv_bfloat16 *>(a.q);
     const __nv_bfloat16 *kg = static_cast<const __nv_bfloat16 *>(a.k);
@@ -140,7 +145,7 @@ __device__ __noinline__ void exact_diag_channel(const KdaChunkArgs &a, int64_t c
             const size_t off = ((size_t)(c0 + R) * H + h) * DK + ch;
             if (R > I) f *= __expf(a.log_alpha[off]);
             const float kd = ki * f;
-            if (R > I) atomicAdd(&Am[R * LF + I], sBeta[R] * __bfloat162float(kg[off]) * kd);
+            if (R > I) atomicAdd(&sCA[blk * 256 + (R - 16 * blk) * 16 + i], sBeta[R] * __bfloat162float(kg[off]) * kd);
             atomicAdd(&sCP[blk * 256 + (R - 16 * blk) * 16 + i], a.scale * __bfloat162float(qg[off]) * kd);
         }
     }
@@ -182,7 +187,7 @@ __global__ void __launch_bounds__(NTHR, 2)
 
     uint8_t *sKQ = sm + I_KQ, *sKC = sm + I_KC, *sIP = sm + I_KC, *sTP = sm + I_TP;
     float *Am = (float *)(sm + I_AM), *Tm = (float *)(sm + I_TM);
-    float *sSC = (float *)(sm + I_SC), *sCP = (float *)(sm + I_CP);
+    float *sSC = (float *)(sm + I_SC), *sCP = (float *)(sm + I_CP), *sCA = (float *)(sm + I_CA);
     float *sBeta = (float *)(sm + I_BETA), *sGC = (float *)(sm + I_GC);
     float *sBS = (float *)(sm + I_BS), *sBT = (float *)(sm + I_BT), *sXT = (float *)(sm + I_XT);
     const float scale = a.scale;
@@ -201,14 +206,15 @@ __global__ void __launch_bounds__(NTHR, 2)
         la[rr] = ok ? *reinterpret_cast<const float2 *>(a.log_alpha + off) : make_float2(0.f, 0.f);
         kr2[rr] = ok ? *reinterpret_cast<const uint32_t *>(kg + off) : 0u;
     }
-    // q goes to shared memory (row-major [64][128] in the space of [T'; P T'], unused until
-    // then), which keeps it out of the registers; rows past the chunk's end are zero-filled.
+    // q goes to shared memory (a [64][128] tile in the rm_sw layout, in the space of
+    // [T'; P T'], unused until then), which keeps it out of the registers; rows past the
+    // chunk's end are zero-filled.
     uint8_t *sQ = sTP;
 #pragma unroll
     for (int k4 = 0; k4 < 4; ++k4) {
         const int idx = tid + NTHR * k4, r = idx >> 4, j = idx & 15;
         const bool ok = r < nr;
-        cp_async16(sQ + r * 256 + 16 * j, ok ? qg + ((size_t)(c0 + r) * H + h) * DK + 8 * j : qg, ok ? 16u : 0u);
+        cp_async16(sQ + rm_sw(r, 8 * j), ok ? qg + ((size_t)(c0 + r) * H + h) * DK + 8 * j : qg, ok ? 16u : 0u);
     }
     if (tid < CH) sBeta[tid] = tid < nr ? a.beta[(size_t)(c0 + tid) * H + h] : 0.f;
 
@@ -224,8 +230,8 @@ __global__ void __launch_bounds__(NTHR, 2)
     // ---------------- E2 pass 1: alpha, per-block sums and products; clear the exact-path sums
 #pragma unroll
     for (int k4 = 0; k4 < 4; ++k4) {
-        const int idx = tid + NTHR * k4, blk = idx >> 8;
-        Am[(16 * blk + ((idx >> 4) & 15)) * LF + 16 * blk + (idx & 15)] = 0.f;
+        const int idx = tid + NTHR * k4;
+        sCA[idx] = 0.f;
         sCP[idx] = 0.f;
     }
     {
@@ -278,8 +284,9 @@ __global__ void __launch_bounds__(NTHR, 2)
         const bool fl0 = bs.x < -kSpreadLimit, fl1 = bs.y < -kSpreadLimit;
         const float rho0 = fast || fl0 ? 1.f : __expf(-0.5f * bs.x);
         const float rho1 = fast || fl1 ? 1.f : __expf(-0.5f * bs.y);
-        __nv_bfloat16 *gKL = (__nv_bfloat16 *)(gslot + SLOT_KL), *gKR = (__nv_bfloat16 *)(gslot + SLOT_KR);
-        __nv_bfloat16 *gQL = (__nv_bfloat16 *)(gslot + SLOT_QL);
+        // the block path's factors, rm_sw tiles: left k in the space of A, right k in the space of
+        // k e^-g / [I; P], left s q in place of q (each thread rewrites the elements it read)
+        uint8_t *sKL = sm + I_AM, *sKR = sm + I_KC;
         if (fast) {
             float l0 = 1.f, l1 = 1.f;
 #pragma unroll
@@ -287,7 +294,7 @@ __global__ void __launch_bounds__(NTHR, 2)
                 const int r = 16 * eb + rr;
                 l0 *= la[rr].x;
                 l1 *= la[rr].y;
-                const float2 kv = unpack_bf16(kr2[rr]), qv = unpack_bf16(*(const uint32_t *)(sQ + r * 256 + 2 * c2));
+                const float2 kv = unpack_bf16(kr2[rr]), qv = unpack_bf16(*(const uint32_t *)(sQ + rm_sw(r, c2)));
                 const float g0 = gpre.x * l0, g1 = gpre.y * l1;
                 *(uint32_t *)(sKQ + col_kq + sw128(r, c2 & 63)) = pack_bf16(kv.x * g0, kv.y * g1);
                 *(uint32_t *)(sKQ + col_kq + sw128(64 + r, c2 & 63)) = pack_bf16(scale * qv.x * g0, scale * qv.y * g1);
@@ -309,12 +316,12 @@ __global__ void __launch_bounds__(NTHR, 2)
                 const int r = 16 * eb + rr;
                 l0 *= la[rr].x;
                 l1 *= la[rr].y;
-                const float2 kv = unpack_bf16(kr2[rr]), qv = unpack_bf16(*(const uint32_t *)(sQ + r * 256 + 2 * c2));
+                const float2 kv = unpack_bf16(kr2[rr]), qv = unpack_bf16(*(const uint32_t *)(sQ + rm_sw(r, c2)));
                 const float g0 = gpre.x * l0, g1 = gpre.y * l1;
                 *(uint32_t *)(sKQ + col_kq + sw128(r, c2 & 63)) = pack_bf16(kv.x * g0, kv.y * g1);
                 *(uint32_t *)(sKQ + col_kq + sw128(64 + r, c2 & 63)) = pack_bf16(scale * qv.x * g0, scale * qv.y * g1);
-                *(uint32_t *)&gKL[r * 128 + c2] = pack_bf16(kv.x * (rho0 * l0), kv.y * (rho1 * l1));
-                *(uint32_t *)&gQL[r * 128 + c2] =
+                *(uint32_t *)(sKL + rm_sw(r, c2)) = pack_bf16(kv.x * (rho0 * l0), kv.y * (rho1 * l1));
+                *(uint32_t *)(sQ + rm_sw(r, c2)) =
                     pack_bf16(scale * qv.x * (rho0 * l0), scale * qv.y * (rho1 * l1));
             }
             float g0 = 1.f, g1 = 1.f;
@@ -324,13 +331,13 @@ __global__ void __launch_bounds__(NTHR, 2)
                 const float2 kv = unpack_bf16(kr2[rr]);
                 *(uint32_t *)(gslot + SLOT_KC + col_kc + sw128(r, c2 & 63)) =
                     pack_bf16(kv.x * (g0 * ksuf.x), kv.y * (g1 * ksuf.y));
-                *(uint32_t *)&gKR[r * 128 + c2] = pack_bf16(kv.x * (rho0 * g0), kv.y * (rho1 * g1));
+                *(uint32_t *)(sKR + rm_sw(r, c2)) = pack_bf16(kv.x * (rho0 * g0), kv.y * (rho1 * g1));
                 g0 *= la[rr].x;
                 g1 *= la[rr].y;
             }
         }
-        if (!fast && fl0) exact_diag_channel(a, c0, nr, h, eb, c2, sBeta, Am, sCP);
-        if (!fast && fl1) exact_diag_channel(a, c0, nr, h, eb, c2 + 1, sBeta, Am, sCP);
+        if (!fast && fl0) exact_diag_channel(a, c0, nr, h, eb, c2, sBeta, sCA, sCP);
+        if (!fast && fl1) exact_diag_channel(a, c0, nr, h, eb, c2 + 1, sBeta, sCA, sCP);
         if (eb == 0) {
             float2 gc = make_float2(1.f, 1.f);
 #pragma unroll
@@ -403,43 +410,58 @@ __global__ void __launch_bounds__(NTHR, 2)
             for (int m = 0; m < 4; ++m) *(uint4 *)(sIP + sw128_chunk(trow, 4 * half + m)) = pack8(v + 8 * m);
         }
     } else {
-        // 16 x 16 blocks with block-local decay references, warp MMAs; operands from the slot.
-        const __nv_bfloat16 *gKL = (const __nv_bfloat16 *)(gslot + SLOT_KL);
-        const __nv_bfloat16 *gKR = (const __nv_bfloat16 *)(gslot + SLOT_KR);
-        const __nv_bfloat16 *gQL = (const __nv_bfloat16 *)(gslot + SLOT_QL);
+        // 16 x 16 blocks with block-local decay references, warp MMAs on the factors in shared
+        // memory.  The results stay in registers until every task has read the factors (A and
+        // [I; P] take their space), then go out after a barrier.
+        const uint8_t *sKL = sm + I_AM, *sKR = sm + I_KC;
         const int g = lane >> 2, t4 = lane & 3;
-        for (int task = warp; task < 20; task += 8) {
+        float res[3][2][4];
+#pragma unroll
+        for (int it = 0; it < 3; ++it) {
+            const int task = warp + 8 * it;
+            if (task >= 20) break;
             const int mat = task / 10, p = task % 10, pa = kPairA[p], pb = kPairB[p];
-            const __nv_bfloat16 *Ls = mat == 0 ? gKL : gQL;
+            const uint8_t *Ls = mat == 0 ? sKL : sQ;
             float acc[2][2][4] = {};
 #pragma unroll 2
             for (int kt = 0; kt < 8; ++kt) {
                 const int c = 16 * kt + 2 * t4;
-                const uint32_t a0 = *(const uint32_t *)&Ls[(16 * pa + g) * 128 + c];
-                const uint32_t a1 = *(const uint32_t *)&Ls[(16 * pa + g + 8) * 128 + c];
-                const uint32_t a2 = *(const uint32_t *)&Ls[(16 * pa + g) * 128 + c + 8];
-                const uint32_t a3 = *(const uint32_t *)&Ls[(16 * pa + g + 8) * 128 + c + 8];
+                const uint32_t a0 = *(const uint32_t *)(Ls + rm_sw(16 * pa + g, c));
+                const uint32_t a1 = *(const uint32_t *)(Ls + rm_sw(16 * pa + g + 8, c));
+                const uint32_t a2 = *(const uint32_t *)(Ls + rm_sw(16 * pa + g, c + 8));
+                const uint32_t a3 = *(const uint32_t *)(Ls + rm_sw(16 * pa + g + 8, c + 8));
                 const float2 s01 = *reinterpret_cast<const float2 *>(&sSC[p * 128 + c]);
                 const float2 s89 = *reinterpret_cast<const float2 *>(&sSC[p * 128 + c + 8]);
 #pragma unroll
                 for (int j = 0; j < 2; ++j) {
                     const int i = 16 * pb + 8 * j + g;
-                    const float2 f0 = unpack_bf16(*(const uint32_t *)&gKR[i * 128 + c]);
-                    const float2 f1 = unpack_bf16(*(const uint32_t *)&gKR[i * 128 + c + 8]);
+                    const float2 f0 = unpack_bf16(*(const uint32_t *)(sKR + rm_sw(i, c)));
+                    const float2 f1 = unpack_bf16(*(const uint32_t *)(sKR + rm_sw(i, c + 8)));
                     mma_m16n8k16(acc[kt & 1][j], a0, a1, a2, a3, pack_bf16(f0.x * s01.x, f0.y * s01.y),
                                  pack_bf16(f1.x * s89.x, f1.y * s89.y));
                 }
             }
+#pragma unroll
+            for (int j = 0; j < 2; ++j)
+#pragma unroll
+                for (int e = 0; e < 4; ++e) res[it][j][e] = acc[0][j][e] + acc[1][j][e];
+        }
+        __syncthreads();
+#pragma unroll
+        for (int it = 0; it < 3; ++it) {
+            const int task = warp + 8 * it;
+            if (task >= 20) break;
+            const int mat = task / 10, p = task % 10, pa = kPairA[p], pb = kPairB[p];
 #pragma unroll
             for (int j = 0; j < 2; ++j) {
 #pragma unroll
                 for (int e = 0; e < 4; ++e) {
                     const int r = 16 * pa + g + (e >= 2 ? 8 : 0);
                     const int i = 16 * pb + 8 * j + 2 * t4 + (e & 1);
-                    const float val = acc[0][j][e] + acc[1][j][e];
+                    const float val = res[it][j][e];
                     if (mat == 0) {
                         if (pa != pb) Am[r * LF + i] = sBeta[r] * val;
-                        else if (i < r) Am[r * LF + i] += sBeta[r] * val;
+                        else if (i < r) Am[r * LF + i] = sBeta[r] * val + sCA[pa * 256 + (r & 15) * 16 + (i & 15)];
                     } else {
                         float pv = val;
                         if (pa == pb) pv = i <= r ? pv + sCP[pa * 256 + (r & 15) * 16 + (i & 15)] : 0.f;
