@@ -115,17 +115,42 @@ __device__ __forceinline__ uint32_t rm_sw(int r, int c) {
     return (uint32_t)(r * 256 + (((c >> 3) ^ (r & 7)) << 4) + ((c & 7) << 1));
 }
 
-// Slot bases of the sequences: base[n] = sum_{m<n} ceil(len_m / 64).
-__global__ void kda_chunk_slots_kernel(const int32_t *cu_seqlens, int N, int64_t T_total, int32_t *base) {
-    if (threadIdx.x != 0) return;
-    int32_t acc = 0;
-    for (int n = 0; n < N; ++n) {
-        int64_t t0, t1;
-        kda::seq_bounds(cu_seqlens, n, 0, T_total, t0, t1);
-        base[n] = acc;
-        acc += (int32_t)((t1 - t0 + CH - 1) / CH);
+// Varlen bookkeeping in the workspace head: base[n] = sum_{m<n} ceil(len_m / 64) (the slot
+// offsets), and order[0..N) = the sequences by decreasing length (ties by index), so the scan
+// starts its longest chains first.  Up to kSortMax sequences are ranked; beyond that the order
+// is the identity.
+constexpr int kSortMax = 256;
+
+__global__ void __launch_bounds__(kSortMax) kda_chunk_slots_kernel(const int32_t *cu_seqlens, int N,
+                                                                    int64_t T_total, int32_t *base,
+                                                                    int32_t *order) {
+    if (threadIdx.x == 0) {
+        int32_t acc = 0;
+        for (int n = 0; n < N; ++n) {
+            int64_t t0, t1;
+            kda::seq_bounds(cu_seqlens, n, 0, T_total, t0, t1);
+            base[n] = acc;
+            acc += (int32_t)((t1 - t0 + CH - 1) / CH);
+        }
+        base[N] = acc;
     }
-    base[N] = acc;
+    if (N > kSortMax) {
+        for (int n = threadIdx.x; n < N; n += blockDim.x) order[n] = n;
+        return;
+    }
+    __shared__ int64_t len[kSortMax];
+    const int t = threadIdx.x;
+    if (t < N) {
+        int64_t t0, t1;
+        kda::seq_bounds(cu_seqlens, t, 0, T_total, t0, t1);
+        len[t] = t1 - t0;
+    }
+    __syncthreads();
+    if (t < N) {
+        int rank = 0;
+        for (int m = 0; m < N; ++m) rank += (len[m] > len[t] || (len[m] == len[t] && m < t)) ? 1 : 0;
+        order[rank] = t;
+    }
 }
 
 // Exact diagonal-block contribution of one channel whose decay over a 16-row block is too
@@ -694,8 +719,13 @@ __global__ void __launch_bounds__(SCAN_THREADS, 1)
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int H = a.H;
-    const int pair = blockIdx.x / NTILE, tile = blockIdx.x % NTILE;
-    const int n = pair / H, h = pair % H;
+    // Varlen: CTAs walk the sequences longest first (the order the slot kernel wrote after the
+    // slot offsets); fixed length: in index order.
+    const int rank = blockIdx.x / (H * NTILE), rest = blockIdx.x % (H * NTILE);
+    const int h = rest / NTILE, tile = rest % NTILE;
+    int n = slot_base ? slot_base[a.N + 1 + rank] : rank;
+    if (n < 0 || n >= a.N) n = 0;             // not reached: the order is a permutation
+    const int pair = n * H + h;
     __nv_bfloat16 *og = static_cast<__nv_bfloat16 *>(a.out);
     int64_t t0, t1;
     kda::seq_bounds(a.cu_seqlens, n, a.T, a.T_total, t0, t1);
@@ -1007,8 +1037,8 @@ cudaError_t encode_tok_map(const KdaChunkArgs &a, const void *base, CUtensorMap 
 int64_t max_slots_of(const KdaChunkArgs &a) {
     return a.cu_seqlens ? (a.T_total + CH - 1) / CH + a.N : (int64_t)a.N * ((a.T + CH - 1) / CH);
 }
-size_t head_bytes_of(const KdaChunkArgs &a) {
-    return ((size_t)(a.N + 1) * sizeof(int32_t) + 1023) & ~(size_t)1023;
+size_t head_bytes_of(const KdaChunkArgs &a) {      // slot offsets [N + 1], order [N]
+    return ((size_t)(2 * a.N + 1) * sizeof(int32_t) + 1023) & ~(size_t)1023;
 }
 
 }  // namespace
@@ -1028,7 +1058,9 @@ cudaError_t kda_launch_chunk_tc_ws(const KdaChunkArgs &a, void *ws, cudaStream_t
     int32_t *slot_base = a.cu_seqlens ? static_cast<int32_t *>(ws) : nullptr;
     uint8_t *slots = static_cast<uint8_t *>(ws) + head_bytes_of(a);
     if (max_slots > 0) {
-        if (a.cu_seqlens) kda_chunk_slots_kernel<<<1, 32, 0, stream>>>(a.cu_seqlens, a.N, a.T_total, slot_base);
+        if (a.cu_seqlens)
+            kda_chunk_slots_kernel<<<1, kSortMax, 0, stream>>>(a.cu_seqlens, a.N, a.T_total, slot_base,
+                                                                slot_base + a.N + 1);
         const dim3 grid((unsigned)max_slots, (unsigned)a.H);
         kda_chunk_intra_kernel<<<grid, NTHR, kIntraSmem, stream>>>(a, slots, slot_base);
     }

@@ -88,9 +88,10 @@ enum kda_status {
  * Empty sequences (and T = 0) are allowed: their S_final is S0 (or zero).
  * Workspace: with KDA_BF16 and dk = dv = 128 the call runs two kernels (one per
  * (chunk, head), then one scan per (sequence, head)) that hand each chunk's operands
- * over through a device workspace of 66,560 bytes per (chunk, head) plus 4 (N + 1)
- * bytes, rounded up to 1 KiB.  It is taken with cudaMallocAsync on `stream` from the
- * device's default memory pool and returned with cudaFreeAsync on the same stream;
+ * over through a device workspace of 66,560 bytes per (chunk, head) plus 4 (2N + 1)
+ * bytes (slot offsets and the scan order), rounded up to 1 KiB.  It is taken with
+ * cudaMallocAsync on `stream` from the device's default memory pool and returned with
+ * cudaFreeAsync on the same stream;
  * the pool's release threshold is raised on first use so the memory stays in the
  * pool between calls.  Every other dtype and size allocates nothing.
  * Supported sizes: KDA_F32 any dk, dv in {32, 64, 128}; KDA_BF16 dk = dv = 128, or
@@ -116,7 +117,7 @@ int kda_chunk_fwd(const void *q, const void *k, const void *v, const float *log_
  * KDA_ERR_SCRATCH.  Where kda_chunk_fwd takes its workspace from the memory pool,
  * this call uses a buffer of KDA_NOALLOC_SCRATCH_BYTES (64 MiB) that is part of the
  * library's device image, one per device; no allocator (CUDA's or any other) is called.
- *  - Limit: the workspace must fit: 66,560 bytes per (chunk, head) plus 4 (N + 1)
+ *  - Limit: the workspace must fit: 66,560 bytes per (chunk, head) plus 4 (2N + 1)
  *    bytes rounded up to 1 KiB, counting ceil(T / 64) chunks per sequence without
  *    cu_seqlens and ceil(T / 64) + N chunks in all with it.  That is at most 1,008
  *    (chunk, head) pairs, e.g. one 4,032-token sequence with 16 heads.  A larger
