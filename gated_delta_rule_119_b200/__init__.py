@@ -2,7 +2,9 @@
 C ABI of libkda.so (include/kda.h).  Importing the package does not load the
 library; the first call does, and fails loudly if it is missing."""
 from .binding import (KDA_BF16, KDA_F32, KDAError, kda_chunk_fwd, kda_decode_step,
-                      kda_device_status, kda_status_string, load_library)
+                      kda_device_status, kda_selftest_wait_timeout, kda_status_string,
+                      load_library)
 
 __all__ = ["KDA_BF16", "KDA_F32", "KDAError", "kda_chunk_fwd", "kda_decode_step",
-           "kda_device_status", "kda_status_string", "load_library"]
+           "kda_device_status", "kda_selftest_wait_timeout", "kda_status_string",
+           "load_library"]

@@ -17,7 +17,7 @@ STATUS = {0: "KDA_OK", -1: "KDA_ERR_NULL", -2: "KDA_ERR_DIM", -3: "KDA_ERR_CHUNK
           -4: "KDA_ERR_ALIGN", -5: "KDA_ERR_DTYPE", -6: "KDA_ERR_ALIAS", -7: "KDA_ERR_CUDA",
           -8: "KDA_ERR_TIMEOUT", -9: "KDA_ERR_SCRATCH"}
 EXPORTS = ("kda_chunk_fwd", "kda_chunk_fwd_noalloc", "kda_decode_step", "kda_device_status",
-           "kda_status_string")
+           "kda_selftest_wait_timeout", "kda_status_string")
 NOALLOC_SCRATCH_BYTES = 64 * 1024 * 1024   # KDA_NOALLOC_SCRATCH_BYTES
 
 _lib = None
@@ -46,6 +46,8 @@ def load_library(path: str | None = None):
     lib.kda_chunk_fwd_noalloc.restype = ctypes.c_int
     lib.kda_decode_step.argtypes = [V, V, V, F, F, F, V] + [I32] * 5 + [V]
     lib.kda_decode_step.restype = ctypes.c_int
+    lib.kda_selftest_wait_timeout.argtypes = [I32, V]
+    lib.kda_selftest_wait_timeout.restype = ctypes.c_int
     lib.kda_device_status.argtypes = []
     lib.kda_device_status.restype = ctypes.c_int
     lib.kda_status_string.argtypes = [ctypes.c_int]
@@ -59,6 +61,12 @@ def kda_device_status() -> int:
     """Synchronise the device; KDA_ERR_TIMEOUT (-8) if a kernel gave up a bounded
     wait since the previous call, else 0.  Clears the record."""
     return load_library().kda_device_status()
+
+
+def kda_selftest_wait_timeout(limit_us: int, stream: int = 0) -> int:
+    """Launch the bounded-wait self-test (one thread waits on an mbarrier nothing arrives at
+    for about `limit_us` microseconds, then records a timeout).  Returns the launch status."""
+    return load_library().kda_selftest_wait_timeout(int(limit_us), stream or None)
 
 
 def kda_status_string(status: int) -> str:

@@ -146,6 +146,11 @@ extern "C" int kda_decode_step(const void *q, const void *k, const void *v, cons
     return cuda_status(kda_launch_decode(a, dtype, reinterpret_cast<cudaStream_t>(stream)));
 }
 
+extern "C" int kda_selftest_wait_timeout(int limit_us, kda_stream_t stream) {
+    if (limit_us < 1 || limit_us > 1000000) return KDA_ERR_DIM;
+    return cuda_status(kda_launch_wait_selftest(limit_us, reinterpret_cast<cudaStream_t>(stream)));
+}
+
 extern "C" int kda_device_status(void) {
     unsigned int st = 0;
     const cudaError_t e = kda_read_device_status(&st, true);

@@ -1085,6 +1085,27 @@ cudaError_t kda_launch_chunk_tc(const KdaChunkArgs &a, cudaStream_t stream) {
     return e != cudaSuccess ? e : f;
 }
 
+// Self-test of the bounded device waits: one thread waits on an mbarrier that nothing arrives
+// at, gives up after `limit_cycles` SM clock cycles and records the timeout the way the prefill
+// kernels do, so that kda_device_status() reports it and the context stays usable.
+__global__ void kda_wait_selftest_kernel(long long limit_cycles) {
+    __shared__ uint64_t bar;
+    if (threadIdx.x != 0) return;
+    mbar_init(&bar, 1);
+    mbar_init_fence();
+    if (!mbar_wait(&bar, 0, limit_cycles)) atomicOr(&g_kda_device_status, 1u);
+}
+
+cudaError_t kda_launch_wait_selftest(int limit_us, cudaStream_t stream) {
+    int dev = 0, khz = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    if ((e = cudaDeviceGetAttribute(&khz, cudaDevAttrClockRate, dev)) != cudaSuccess) return e;
+    const long long cycles = (long long)limit_us * (khz > 0 ? khz : 2000000) / 1000;
+    kda_wait_selftest_kernel<<<1, 32, 0, stream>>>(cycles);
+    return cudaGetLastError();
+}
+
 cudaError_t kda_read_device_status(unsigned int *status, bool clear) {
     cudaError_t e = cudaDeviceSynchronize();
     if (e != cudaSuccess) return e;

@@ -68,3 +68,4 @@ cudaError_t kda_launch_chunk_tc_ws(const KdaChunkArgs &a, void *ws, cudaStream_t
 // Device address of the fixed scratch buffer of the current device (kda_noalloc.cu).
 cudaError_t kda_noalloc_scratch(void **ptr);
 cudaError_t kda_read_device_status(unsigned int *status, bool clear);
+cudaError_t kda_launch_wait_selftest(int limit_us, cudaStream_t stream);

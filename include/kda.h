@@ -166,6 +166,17 @@ int kda_decode_step(const void *q, const void *k, const void *v, const float *lo
  */
 int kda_device_status(void);
 
+/*
+ * kda_selftest_wait_timeout -- exercises the bounded-wait machinery without a fault.  The
+ * pages have no counterpart of this call.  It launches one thread on `stream` that waits on
+ * an mbarrier nothing arrives at; after about `limit_us` microseconds of SM clock it gives up
+ * and records a timeout exactly as the prefill kernels do when one of their waits runs out.
+ * The next kda_device_status() then returns KDA_ERR_TIMEOUT and clears the record; the CUDA
+ * context stays usable.  limit_us must be in [1, 1000000] (else KDA_ERR_DIM).
+ * Returns KDA_OK or KDA_ERR_CUDA (launch failure).
+ */
+int kda_selftest_wait_timeout(int limit_us, kda_stream_t stream);
+
 /* A static, human-readable description of a status code.  For KDA_ERR_CUDA it names
  * the CUDA error of the calling host thread's last failed launch. */
 const char *kda_status_string(int status);

@@ -91,3 +91,8 @@ def test_decode_step_rejects(lib, kw, code):
 def test_product_path_fails_loudly_without_library(tmp_path):
     with pytest.raises(RuntimeError, match="libkda.so not found"):
         binding.load_library(str(tmp_path / "libkda.so"))
+
+
+@pytest.mark.parametrize("limit_us", [0, -5, 1000001])
+def test_wait_selftest_rejects_out_of_range_limits(lib, limit_us):
+    assert binding.kda_selftest_wait_timeout(limit_us) == -2      # KDA_ERR_DIM, before any CUDA call

@@ -89,3 +89,20 @@ def test_sequence_split_across_calls(dtype):
     eo, es = rel_err(o, ro), rel_err(s2.cpu().numpy(), rs)
     print(f"[behaviour] split {dtype}: o {eo:.3e}  S_final {es:.3e}")
     assert eo <= TOL[dtype] and es <= TOL[dtype]
+
+
+def test_bounded_wait_selftest_reports_timeout_and_context_survives():
+    """A wait that nothing ends gives up after its limit: kda_device_status() reports
+    KDA_ERR_TIMEOUT once, then clears, and the next prefill still runs and matches."""
+    from gated_delta_rule_119_b200 import kda_device_status, kda_selftest_wait_timeout
+    assert kda_device_status() == 0
+    assert kda_selftest_wait_timeout(2000) == 0
+    assert kda_device_status() == -8
+    assert kda_device_status() == 0
+    inp = make_inputs(1, 200, 2, 128, 128, "bf16", 1205, state=True)
+    o, s = call(to_torch(inp))
+    torch.cuda.synchronize()
+    ro, rs = oracle.recurrent_full(inp.q, inp.k, inp.v, inp.log_alpha, inp.beta, inp.S0, inp.offsets())
+    o = o.float().cpu().numpy().reshape(inp.total_tokens, inp.H, inp.dv)
+    assert rel_err(o, ro) <= TOL["bf16"] and rel_err(s.cpu().numpy(), rs) <= TOL["bf16"]
+    assert kda_device_status() == 0
