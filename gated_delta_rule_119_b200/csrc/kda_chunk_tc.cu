@@ -17,9 +17,10 @@
 // nothing in it depends on the state -- and writes the chunk's tensor-core operands
 // [T'; P T'], [-W; s q gamma - P W], the update operand and gamma_last into one
 // workspace slot, already in the shared-memory image the tensor core reads.  The scan
-// kernel walks each (sequence, head, 64-column slice of d_v) chunk by chunk: it
-// bulk-copies the next slot while the current chunk runs, and per chunk only reads the
-// state out of tensor memory, forms [u; o] and updates the state.
+// kernel walks each (sequence, head, 64-column slice of d_v) chunk by chunk with
+// specialised warps: one fetches the next slot (bulk copy) and v tile (TMA) while the
+// current chunk runs, one issues the tensor-core products, eight move the state, u and o
+// through tensor memory, and one stores o (TMA).
 //
 // Intra-chunk kernel, per (chunk, head):
 //  E2  one thread per (2 channels, 16-row block): alpha = exp(log_alpha), block-local
@@ -33,7 +34,8 @@
 //      an exact per-channel path for blocks whose spread exceeds that range, and the
 //      update operand k kappa.
 //  T   T = (I + A)^{-1}: 16 x 16 diagonal blocks by substitution in fp32, the rest with
-//      tf32 warp MMAs; [T'; P T'] = [I; P] T' and [W; P W] = [T'; P T'] (k gamma) on tcgen05.
+//      tf32 warp MMAs; [T'; P T'] = [I; P] T' and
+//      [-W; s q gamma - P W] = [0; s q gamma] - [T'; P T'] (k gamma) on tcgen05.
 #include <cuda.h>
 #include <cudaTypedefs.h>
 #include <stdio.h>
@@ -692,7 +694,7 @@ __global__ void __launch_bounds__(NTHR, 2)
 // TMEM for the whole sequence.  Warp roles, joined only through mbarriers:
 //   warps 0-7  read-out: per chunk c, S out of TMEM (pending decay applied, bf16 copy for the
 //              product), then [u; o] out of TMEM: u into shared memory (warps 0, 1, 4, 5 hold
-//              TMEM lanes 0-63), o to HBM (warps 2, 3, 6, 7);
+//              TMEM lanes 0-63), o into a staging tile for the store thread (warps 2, 3, 6, 7);
 //   warp 8     tensor-core issue (one thread): [u; o] = [T'; P T'] v as soon as the chunk is in
 //              shared memory, + [-W; s q gamma - P W] S once S is copied, S += KC^T u once u is;
 //   warp 9     loads (one thread): slot c and the v tile of chunk c into stage c & 1 once the
