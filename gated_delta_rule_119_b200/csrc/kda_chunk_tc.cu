@@ -187,6 +187,9 @@ __global__ void __launch_bounds__(NTHR, 2)
     __shared__ uint32_t s_tmem;
     __shared__ int s_abort;
 
+    // The scan may be scheduled once every CTA of this grid has started (it waits for this
+    // grid's completion before it reads the workspace).
+    asm volatile("griddepcontrol.launch_dependents;");
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int H = a.H, h = blockIdx.y;
     const int slot = blockIdx.x;
@@ -783,6 +786,8 @@ __global__ void __launch_bounds__(SCAN_THREADS, 1)
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
+    // Everything above runs while the intra-chunk grid finishes; the workspace is read below.
+    asm volatile("griddepcontrol.wait;" ::: "memory");
 
     if (warp == 9) {
         // ------------------------------------------------------------------ loads
@@ -1069,8 +1074,22 @@ cudaError_t kda_launch_chunk_tc_ws(const KdaChunkArgs &a, void *ws, cudaStream_t
     CUtensorMap tmap_v, tmap_o;
     if ((e = encode_tok_map(a, a.v, &tmap_v)) != cudaSuccess) return e;
     if ((e = encode_tok_map(a, a.out, &tmap_o)) != cudaSuccess) return e;
-    kda_chunk_scan_kernel<<<(unsigned)((int64_t)a.N * a.H * NTILE), SCAN_THREADS, kScanSmem, stream>>>(
-        a, slots, slot_base, tmap_v, tmap_o);
+    // Launched with programmatic stream serialisation: its CTAs may start (barrier set-up, TMEM
+    // allocation, S0 into TMEM) while the last intra-chunk CTAs run; the kernel waits for
+    // that grid before it reads the workspace.
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)((int64_t)a.N * a.H * NTILE));
+    cfg.blockDim = dim3(SCAN_THREADS);
+    cfg.dynamicSmemBytes = kScanSmem;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = max_slots > 0 ? 1 : 0;   // without the intra grid, an ordinary launch
+    if ((e = cudaLaunchKernelEx(&cfg, kda_chunk_scan_kernel, a, static_cast<const uint8_t *>(slots),
+                                static_cast<const int32_t *>(slot_base), tmap_v, tmap_o)) != cudaSuccess)
+        return e;
     return cudaGetLastError();
 }
 
