@@ -41,6 +41,8 @@
 #include <stdio.h>
 #include <string.h>
 
+#include <atomic>
+
 #include "kda_common.cuh"
 #include "kda_tc_util.cuh"
 
@@ -983,32 +985,36 @@ __global__ void __launch_bounds__(SCAN_THREADS, 1)
     if (warp == 0) tmem_free(tmem, 256);
 }
 
-bool g_configured[64] = {};
+// Per-device "already done" flags of the one-time set-up below.  Host threads may call the
+// library concurrently: a flag is only a shortcut (the set-up calls are idempotent), so two
+// threads that both find it clear both run the set-up, which is harmless.
+constexpr int kMaxDevices = 64;
+std::atomic<bool> g_configured[kMaxDevices] = {};
+std::atomic<bool> g_pool_configured[kMaxDevices] = {};
 
 cudaError_t configure(int dev) {
-    if (dev >= 0 && dev < 64 && g_configured[dev]) return cudaSuccess;
+    if (dev >= 0 && dev < kMaxDevices && g_configured[dev].load(std::memory_order_acquire)) return cudaSuccess;
     cudaError_t e = cudaFuncSetAttribute(kda_chunk_intra_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)kIntraSmem);
     if (e != cudaSuccess) return e;
     e = cudaFuncSetAttribute(kda_chunk_scan_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kScanSmem);
     if (e != cudaSuccess) return e;
-    if (dev >= 0 && dev < 64) g_configured[dev] = true;
+    if (dev >= 0 && dev < kMaxDevices) g_configured[dev].store(true, std::memory_order_release);
     return cudaSuccess;
 }
-
-bool g_pool_configured[64] = {};
 
 // Keep freed workspace in the device's default pool between calls instead of returning
 // it to the driver.
 cudaError_t configure_pool(int dev) {
-    if (dev >= 0 && dev < 64 && g_pool_configured[dev]) return cudaSuccess;
+    if (dev >= 0 && dev < kMaxDevices && g_pool_configured[dev].load(std::memory_order_acquire))
+        return cudaSuccess;
     cudaMemPool_t pool;
     cudaError_t e = cudaDeviceGetDefaultMemPool(&pool, dev);
     if (e != cudaSuccess) return e;
     uint64_t keep = ~0ull;
     e = cudaMemPoolSetAttribute(pool, cudaMemPoolAttrReleaseThreshold, &keep);
     if (e != cudaSuccess) return e;
-    if (dev >= 0 && dev < 64) g_pool_configured[dev] = true;
+    if (dev >= 0 && dev < kMaxDevices) g_pool_configured[dev].store(true, std::memory_order_release);
     return cudaSuccess;
 }
 
@@ -1017,27 +1023,28 @@ cudaError_t configure_pool(int dev) {
 // one TMA store writes a chunk's o tile.  Tokens past T_total read as zeros; tokens of the next
 // sequence that fill a partial last chunk of v only meet zero columns of [T'; P T'], and o of a
 // partial chunk is never stored by TMA.
-PFN_cuTensorMapEncodeTiled_v12000 g_encode_tiled = nullptr;
+std::atomic<PFN_cuTensorMapEncodeTiled_v12000> g_encode_tiled{nullptr};
 
 cudaError_t encode_tok_map(const KdaChunkArgs &a, const void *base, CUtensorMap *map) {
     memset(map, 0, sizeof(*map));
     if (a.T_total == 0) return cudaSuccess;       // no chunk: the map is never read
-    if (g_encode_tiled == nullptr) {
+    PFN_cuTensorMapEncodeTiled_v12000 encode = g_encode_tiled.load(std::memory_order_acquire);
+    if (encode == nullptr) {
         void *fn = nullptr;
         cudaDriverEntryPointQueryResult q;
         const cudaError_t e = cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q);
         if (e != cudaSuccess) return e;
         if (q != cudaDriverEntryPointSuccess || fn == nullptr) return cudaErrorNotSupported;
-        g_encode_tiled = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
+        encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
+        g_encode_tiled.store(encode, std::memory_order_release);
     }
     const cuuint64_t dims[3] = {(cuuint64_t)DV, (cuuint64_t)a.H, (cuuint64_t)a.T_total};
     const cuuint64_t strides[2] = {(cuuint64_t)DV * 2, (cuuint64_t)a.H * DV * 2};
     const cuuint32_t box[3] = {(cuuint32_t)DVT, 1, (cuuint32_t)CH};
     const cuuint32_t estr[3] = {1, 1, 1};
-    const CUresult r = g_encode_tiled(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(base), dims,
-                                      strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
-                                      CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-                                      CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    const CUresult r = encode(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(base), dims, strides,
+                              box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
 }
 

@@ -1,7 +1,8 @@
 """GPU behaviour of the C ABI beyond single-call parity: calls on a side stream, run-to-run
 determinism of the tensor-core prefill, many heads with short sequences, one sequence split
-into several calls (S_final fed back as S0).  All through libkda.so; oracle values where a
-value is checked (max|x - r| / max|r| within the dtype's bar)."""
+into several calls (S_final fed back as S0), concurrent calls from several host threads.
+All through libkda.so; oracle values where a value is checked (max|x - r| / max|r| within
+the dtype's bar)."""
 import numpy as np
 import pytest
 
@@ -105,4 +106,46 @@ def test_bounded_wait_selftest_reports_timeout_and_context_survives():
     ro, rs = oracle.recurrent_full(inp.q, inp.k, inp.v, inp.log_alpha, inp.beta, inp.S0, inp.offsets())
     o = o.float().cpu().numpy().reshape(inp.total_tokens, inp.H, inp.dv)
     assert rel_err(o, ro) <= TOL["bf16"] and rel_err(s.cpu().numpy(), rs) <= TOL["bf16"]
+    assert kda_device_status() == 0
+
+
+def test_concurrent_host_threads_match_sequential_calls():
+    """Four host threads, each with its own stream and problem (fixed-length and varlen,
+    bf16 tensor-core path and fp32 SIMT path), call the library at the same time: every
+    result equals the one the same call gives alone.  The ctypes call releases the GIL, so
+    the calls really overlap on the host, set-up included."""
+    import threading
+    cases = [make_inputs(2, 900, 4, 128, 128, "bf16", 1206, state=True),
+             make_inputs(3, 1500, 2, 128, 128, "bf16", 1207, state=True, varlen=True),
+             make_inputs(1, 650, 3, 128, 128, "bf16", 1208, gates="extremes"),
+             make_inputs(2, 300, 2, 64, 64, "f32", 1209, state=True)]
+    data = [to_torch(c) for c in cases]
+    alone = [call(d) for d in data]
+    torch.cuda.synchronize()
+    results, errors = [None] * len(data), []
+    start = threading.Barrier(len(data))
+
+    def worker(i):
+        try:
+            st = torch.cuda.Stream()
+            st.wait_stream(torch.cuda.current_stream())
+            start.wait()
+            with torch.cuda.stream(st):
+                outs = [call(data[i]) for _ in range(3)]
+            st.synchronize()
+            results[i] = outs
+        except Exception as exc:      # reported below, with the thread's case
+            errors.append((i, repr(exc)))
+
+    threads = [threading.Thread(target=worker, args=(i,)) for i in range(len(data))]
+    for t in threads:
+        t.start()
+    for t in threads:
+        t.join(timeout=120)
+    assert not any(t.is_alive() for t in threads)
+    assert not errors, errors
+    for (o_ref, s_ref), outs in zip(alone, results):
+        for o, s in outs:
+            assert torch.equal(o, o_ref) and torch.equal(s, s_ref)
+    from gated_delta_rule_119_b200 import kda_device_status
     assert kda_device_status() == 0
