@@ -150,6 +150,35 @@ def test_full_workload_sampled(name):
     check_against_oracle(inp, tasks=tasks)
 
 
+@pytest.mark.parametrize("dtype,d", [("bf16", 128), ("f32", 32)])
+def test_maximum_head_count(dtype, d):
+    """H = 65,535, the largest head count the library accepts, over two ragged sequences of
+    three tokens in all: the largest grids of both prefill paths run (every (chunk, head)
+    of the intra-chunk kernel, 2 x 65,535 x 2 scan CTAs).  The oracle recomputes sampled
+    (sequence, head) pairs, the last head among them; only their states are copied back."""
+    H = 65535
+    inp = make_inputs(2, 3, H, d, d, dtype, 1210, varlen=True)
+    chunk_fwd, _ = kda()
+    t = to_torch(inp)
+    out, Sf = chunk_fwd(t["q"], t["k"], t["v"], t["log_alpha"], t["beta"], None, t["cu_seqlens"],
+                        output_final_state=True)
+    torch.cuda.synchronize()
+    tasks = sorted(set(sampled_tasks(inp, 6, 1211)) | {(0, H - 1), (1, H - 1), (1, 0)})
+    cu = inp.offsets()
+    o = out.float().cpu().numpy().reshape(inp.total_tokens, H, d)
+    S = {(n, h): Sf[n, h].cpu().numpy() for n, h in tasks}
+    del out, Sf, t
+    torch.cuda.empty_cache()
+    from gated_delta_rule_119_b200 import kda_device_status
+    assert kda_device_status() == 0, "a kernel gave up a bounded wait"
+    outs, sts = oracle.recurrent(inp.q, inp.k, inp.v, inp.log_alpha, inp.beta, None, cu, tasks=tasks)
+    eo = rel_err(np.concatenate([o[cu[n]:cu[n + 1], h].ravel() for n, h in tasks]),
+                 np.concatenate([x.ravel() for x in outs]))
+    es = max(rel_err(S[task], st) for task, st in zip(tasks, sts))
+    print(f"[parity] max heads {dtype} d={d}: o {eo:.3e}  S_final {es:.3e}")
+    assert eo <= TOL[dtype] and es <= TOL[dtype]
+
+
 # ----------------------------------------------------------------------- decode
 @pytest.mark.parametrize("dtype", ["f32", "bf16"])
 @pytest.mark.parametrize("dk,dv", [(128, 128), (32, 32), (64, 128), (128, 64)])
