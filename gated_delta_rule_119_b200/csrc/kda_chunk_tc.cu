@@ -23,6 +23,8 @@
 // through tensor memory, and one stores o (TMA).
 //
 // Intra-chunk kernel, per (chunk, head):
+//  IN  one thread loads the chunk's log_alpha, k and q tiles by TMA into shared memory that
+//      later phases reuse.
 //  E2  one thread per (2 channels, 16-row block): alpha = exp(log_alpha), block-local
 //      running products, and from them k gamma, s q gamma (tensor-core operand) and the
 //      update operand.
@@ -112,11 +114,12 @@ __device__ __forceinline__ uint4 pack8(const float *v) {
     return pk;
 }
 
-// Byte offset of element (r, c) of a [64][128] bf16 row-major tile whose 16-byte chunks are
-// XOR-swizzled by r & 7: conflict-free both for a warp reading 32 consecutive channels of one
+// Byte offset of element (r, c) of a [64][128] bf16 tile stored as two 64-column halves of
+// 128-byte rows, the 16-byte chunks of row r XOR-swizzled by r & 7 (the layout a TMA load with
+// 128-byte swizzle writes): conflict-free both for a warp reading 32 consecutive channels of one
 // row and for the warp-MMA fragment loads (8 rows x 4 column pairs).
 __device__ __forceinline__ uint32_t rm_sw(int r, int c) {
-    return (uint32_t)(r * 256 + (((c >> 3) ^ (r & 7)) << 4) + ((c & 7) << 1));
+    return (uint32_t)((c >> 6) * 8192 + r * 128 + ((((c & 63) >> 3) ^ (r & 7)) << 4) + ((c & 7) << 1));
 }
 
 // Varlen bookkeeping in the workspace head: base[n] = sum_{m<n} ceil(len_m / 64) (the slot
@@ -182,10 +185,12 @@ __device__ __noinline__ void exact_diag_channel(const KdaChunkArgs &a, int64_t c
 
 // ======================================================================= intra-chunk kernel
 __global__ void __launch_bounds__(NTHR, 2)
-    kda_chunk_intra_kernel(KdaChunkArgs a, uint8_t *ws, const int32_t *slot_base) {
+    kda_chunk_intra_kernel(KdaChunkArgs a, uint8_t *ws, const int32_t *slot_base,
+                           const __grid_constant__ CUtensorMap tmap_la, const __grid_constant__ CUtensorMap tmap_k,
+                           const __grid_constant__ CUtensorMap tmap_q) {
     extern __shared__ uint8_t smraw[];
     uint8_t *sm = smraw + ((1024u - (smem_u32(smraw) & 1023u)) & 1023u);   // stays a shared-space pointer
-    __shared__ uint64_t bar_ap, bar_p, bar_w;
+    __shared__ uint64_t bar_ap, bar_p, bar_w, bar_in;
     __shared__ uint32_t s_tmem;
     __shared__ int s_abort;
 
@@ -223,41 +228,42 @@ __global__ void __launch_bounds__(NTHR, 2)
     float *sBeta = (float *)(sm + I_BETA), *sGC = (float *)(sm + I_GC);
     float *sBS = (float *)(sm + I_BS), *sBT = (float *)(sm + I_BT), *sXT = (float *)(sm + I_XT);
     const float scale = a.scale;
-    const __nv_bfloat16 *qg = static_cast<const __nv_bfloat16 *>(a.q);
-    const __nv_bfloat16 *kg = static_cast<const __nv_bfloat16 *>(a.k);
 
-    // E2 thread mapping: channels {c2, c2 + 1} of 16-row block eb.  All loads up front.
+    // The chunk's inputs by TMA, issued by one thread: log_alpha [64][128] fp32 into the space of
+    // [k gamma; s q gamma] and k [64][128] bf16 into the space of the update operand (both
+    // row-major; pass 1 moves them to registers before pass 2 overwrites them), q as two
+    // 64-column halves in the rm_sw layout into the space of [T'; P T'].  Rows past the chunk's
+    // end hold the next tokens (zeros past the last token) and are masked where they are read.
+    uint8_t *sQ = sTP;
+    if (tid == 0) {
+        mbar_init(&bar_ap, 1);
+        mbar_init(&bar_p, 1);
+        mbar_init(&bar_w, 1);
+        mbar_init(&bar_in, 1);
+        mbar_init_fence();
+        s_abort = 0;
+        mbar_arrive_expect_tx(&bar_in, 65536);
+        tma_load_3d(sKQ, &tmap_la, 0, h, (int)c0, &bar_in);
+        tma_load_3d(sKC, &tmap_k, 0, h, (int)c0, &bar_in);
+        tma_load_3d(sQ, &tmap_q, 0, h, (int)c0, &bar_in);
+        tma_load_3d(sQ + 8192, &tmap_q, 64, h, (int)c0, &bar_in);
+    }
+    if (tid < CH) sBeta[tid] = tid < nr ? a.beta[(size_t)(c0 + tid) * H + h] : 0.f;
+    if (warp == 0) tmem_alloc(&s_tmem, 256);
+    __syncthreads();                     // the barriers are initialised before anyone waits
+    if (!mbar_wait(&bar_in, 0, kWaitCycles)) s_abort = 1;
+
+    // E2 thread mapping: channels {c2, c2 + 1} of 16-row block eb.
     const int c2 = 2 * (tid & 63), eb = tid >> 6;
     float2 la[16];
     uint32_t kr2[16];
 #pragma unroll
     for (int rr = 0; rr < 16; ++rr) {
         const int r = 16 * eb + rr;
-        const size_t off = ((size_t)(c0 + r) * H + h) * DK + c2;
         const bool ok = r < nr;
-        la[rr] = ok ? *reinterpret_cast<const float2 *>(a.log_alpha + off) : make_float2(0.f, 0.f);
-        kr2[rr] = ok ? *reinterpret_cast<const uint32_t *>(kg + off) : 0u;
+        la[rr] = ok ? *reinterpret_cast<const float2 *>(sKQ + 4 * (r * DK + c2)) : make_float2(0.f, 0.f);
+        kr2[rr] = ok ? *reinterpret_cast<const uint32_t *>(sKC + 2 * (r * DK + c2)) : 0u;
     }
-    // q goes to shared memory (a [64][128] tile in the rm_sw layout, in the space of
-    // [T'; P T'], unused until then), which keeps it out of the registers; rows past the
-    // chunk's end are zero-filled.
-    uint8_t *sQ = sTP;
-#pragma unroll
-    for (int k4 = 0; k4 < 4; ++k4) {
-        const int idx = tid + NTHR * k4, r = idx >> 4, j = idx & 15;
-        const bool ok = r < nr;
-        cp_async16(sQ + rm_sw(r, 8 * j), ok ? qg + ((size_t)(c0 + r) * H + h) * DK + 8 * j : qg, ok ? 16u : 0u);
-    }
-    if (tid < CH) sBeta[tid] = tid < nr ? a.beta[(size_t)(c0 + tid) * H + h] : 0.f;
-
-    if (tid == 0) {
-        mbar_init(&bar_ap, 1);
-        mbar_init(&bar_p, 1);
-        mbar_init(&bar_w, 1);
-        mbar_init_fence();
-        s_abort = 0;
-    }
-    if (warp == 0) tmem_alloc(&s_tmem, 256);
 
     // ---------------- E2 pass 1: alpha, per-block sums and products; clear the exact-path sums
 #pragma unroll
@@ -280,7 +286,6 @@ __global__ void __launch_bounds__(NTHR, 2)
         *reinterpret_cast<float2 *>(&sBS[eb * 128 + c2]) = make_float2(s0, s1);
         *reinterpret_cast<float2 *>(&sBT[eb * 128 + c2]) = make_float2(p0, p1);
     }
-    cp_async_wait_all();
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
@@ -326,7 +331,8 @@ __global__ void __launch_bounds__(NTHR, 2)
                 const int r = 16 * eb + rr;
                 l0 *= la[rr].x;
                 l1 *= la[rr].y;
-                const float2 kv = unpack_bf16(kr2[rr]), qv = unpack_bf16(*(const uint32_t *)(sQ + rm_sw(r, c2)));
+                const float2 kv = unpack_bf16(kr2[rr]);
+                const float2 qv = unpack_bf16(r < nr ? *(const uint32_t *)(sQ + rm_sw(r, c2)) : 0u);
                 const float g0 = gpre.x * l0, g1 = gpre.y * l1;
                 *(uint32_t *)(sKQ + col_kq + sw128(r, c2 & 63)) = pack_bf16(kv.x * g0, kv.y * g1);
                 *(uint32_t *)(sKQ + col_kq + sw128(64 + r, c2 & 63)) = pack_bf16(scale * qv.x * g0, scale * qv.y * g1);
@@ -348,7 +354,8 @@ __global__ void __launch_bounds__(NTHR, 2)
                 const int r = 16 * eb + rr;
                 l0 *= la[rr].x;
                 l1 *= la[rr].y;
-                const float2 kv = unpack_bf16(kr2[rr]), qv = unpack_bf16(*(const uint32_t *)(sQ + rm_sw(r, c2)));
+                const float2 kv = unpack_bf16(kr2[rr]);
+                const float2 qv = unpack_bf16(r < nr ? *(const uint32_t *)(sQ + rm_sw(r, c2)) : 0u);
                 const float g0 = gpre.x * l0, g1 = gpre.y * l1;
                 *(uint32_t *)(sKQ + col_kq + sw128(r, c2 & 63)) = pack_bf16(kv.x * g0, kv.y * g1);
                 *(uint32_t *)(sKQ + col_kq + sw128(64 + r, c2 & 63)) = pack_bf16(scale * qv.x * g0, scale * qv.y * g1);
@@ -689,7 +696,10 @@ __global__ void __launch_bounds__(NTHR, 2)
         bulk_wait_read_all();
     }
     if (tid == 32) bulk_wait_read_all();
-    if (s_abort && tid == 0) atomicOr(&g_kda_device_status, 1u);
+    if (s_abort && tid == 0) {
+        atomicOr(&g_kda_device_status, 1u);
+        mbar_wait(&bar_in, 0, kWaitCycles);   // the input loads must not land in released memory
+    }
     __syncthreads();
     if (warp == 0) tmem_free(tmem, 256);
 }
@@ -1025,7 +1035,16 @@ cudaError_t configure_pool(int dev) {
 // partial chunk is never stored by TMA.
 std::atomic<PFN_cuTensorMapEncodeTiled_v12000> g_encode_tiled{nullptr};
 
+cudaError_t encode_map(const KdaChunkArgs &a, const void *base, CUtensorMapDataType dtype, uint32_t esize,
+                       uint32_t box_x, CUtensorMapSwizzle swizzle, CUtensorMap *map);
+
 cudaError_t encode_tok_map(const KdaChunkArgs &a, const void *base, CUtensorMap *map) {
+    return encode_map(a, base, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, (uint32_t)DVT, CU_TENSOR_MAP_SWIZZLE_128B, map);
+}
+
+// Tensor map of a [T_total][H][128] token tensor with boxes of box_x elements x 1 head x 64 tokens.
+cudaError_t encode_map(const KdaChunkArgs &a, const void *base, CUtensorMapDataType dtype, uint32_t esize,
+                       uint32_t box_x, CUtensorMapSwizzle swizzle, CUtensorMap *map) {
     memset(map, 0, sizeof(*map));
     if (a.T_total == 0) return cudaSuccess;       // no chunk: the map is never read
     PFN_cuTensorMapEncodeTiled_v12000 encode = g_encode_tiled.load(std::memory_order_acquire);
@@ -1038,13 +1057,14 @@ cudaError_t encode_tok_map(const KdaChunkArgs &a, const void *base, CUtensorMap 
         encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
         g_encode_tiled.store(encode, std::memory_order_release);
     }
+    static_assert(DK == DV, "one token-tensor layout for q, k, log_alpha, v and o");
     const cuuint64_t dims[3] = {(cuuint64_t)DV, (cuuint64_t)a.H, (cuuint64_t)a.T_total};
-    const cuuint64_t strides[2] = {(cuuint64_t)DV * 2, (cuuint64_t)a.H * DV * 2};
-    const cuuint32_t box[3] = {(cuuint32_t)DVT, 1, (cuuint32_t)CH};
+    const cuuint64_t strides[2] = {(cuuint64_t)DV * esize, (cuuint64_t)a.H * DV * esize};
+    const cuuint32_t box[3] = {box_x, 1, (cuuint32_t)CH};
     const cuuint32_t estr[3] = {1, 1, 1};
-    const CUresult r = encode(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(base), dims, strides,
-                              box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-                              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    const CUresult r = encode(map, dtype, 3, const_cast<void *>(base), dims, strides, box, estr,
+                              CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
 }
 
@@ -1072,11 +1092,19 @@ cudaError_t kda_launch_chunk_tc_ws(const KdaChunkArgs &a, void *ws, cudaStream_t
     int32_t *slot_base = a.cu_seqlens ? static_cast<int32_t *>(ws) : nullptr;
     uint8_t *slots = static_cast<uint8_t *>(ws) + head_bytes_of(a);
     if (max_slots > 0) {
+        CUtensorMap tmap_la, tmap_k, tmap_q;
+        if ((e = encode_map(a, a.log_alpha, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, DK, CU_TENSOR_MAP_SWIZZLE_NONE,
+                            &tmap_la)) != cudaSuccess)
+            return e;
+        if ((e = encode_map(a, a.k, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, DK, CU_TENSOR_MAP_SWIZZLE_NONE,
+                            &tmap_k)) != cudaSuccess)
+            return e;
+        if ((e = encode_tok_map(a, a.q, &tmap_q)) != cudaSuccess) return e;
         if (a.cu_seqlens)
             kda_chunk_slots_kernel<<<1, kSortMax, 0, stream>>>(a.cu_seqlens, a.N, a.T_total, slot_base,
                                                                 slot_base + a.N + 1);
         const dim3 grid((unsigned)max_slots, (unsigned)a.H);
-        kda_chunk_intra_kernel<<<grid, NTHR, kIntraSmem, stream>>>(a, slots, slot_base);
+        kda_chunk_intra_kernel<<<grid, NTHR, kIntraSmem, stream>>>(a, slots, slot_base, tmap_la, tmap_k, tmap_q);
     }
     CUtensorMap tmap_v, tmap_o;
     if ((e = encode_tok_map(a, a.v, &tmap_v)) != cudaSuccess) return e;

@@ -1,6 +1,6 @@
 // sm_100a building blocks for the tensor-core chunk path: shared-memory
 // operand layout (128-byte swizzle), UMMA descriptors, tcgen05 MMA / commit /
-// TMEM load-store, mbarriers with bounded waits, cp.async, legacy mma.sync.
+// TMEM load-store, mbarriers with bounded waits, TMA and bulk copies, legacy mma.sync.
 //
 // Operand tiles in shared memory are made of 128-byte "lines" (64 bf16).
 // Eight lines form a 1024-byte swizzle atom in which the 16-byte chunk j of
@@ -192,16 +192,6 @@ __device__ __forceinline__ void tmem_st32(uint32_t taddr, const float *v) {
         "r"(r[29]), "r"(r[30]), "r"(r[31])
         : "memory");
     asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
-}
-
-// 16-byte asynchronous global -> shared copy; src_bytes = 0 writes zeros.
-__device__ __forceinline__ void cp_async16(void *dst_smem, const void *src, uint32_t src_bytes) {
-    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(smem_u32(dst_smem)),
-                 "l"(src), "r"(src_bytes)
-                 : "memory");
-}
-__device__ __forceinline__ void cp_async_wait_all() {
-    asm volatile("cp.async.wait_all;" ::: "memory");
 }
 
 // Warp-level bf16 MMA m16n8k16 with fp32 accumulation.
