@@ -184,9 +184,38 @@ def measured_peaks():
 
 
 # ---------------------------------------------------------------- CPU baseline
-def cpu_baseline(inp, budget_s: float = 12.0):
+PARITY_BAR = {"bf16": 2e-2, "f32": 1e-4}
+
+
+def sample_parity(tasks, outs, states, gpu_pair, dtype: str) -> dict:
+    """Max relative error, max|x - r| / max|r|, of the GPU's o (over the sampled pairs' rows
+    together) and of each final state, against the oracle's results for the same (sequence,
+    head) pairs.  gpu_pair(n, h) -> (o [len, dv], S [dk, dv]).  A failure to read the GPU's
+    result is reported in place of the numbers; it never stops the bench."""
+    try:
+        go, ro, es = [], [], 0.0
+        for (n, h), o_ref, s_ref in zip(tasks, outs, states):
+            o_gpu, s_gpu = gpu_pair(n, h)
+            go.append(np.asarray(o_gpu, dtype=np.float64).ravel())
+            ro.append(np.asarray(o_ref, dtype=np.float64).ravel())
+            s_ref = np.asarray(s_ref, dtype=np.float64)
+            es = max(es, float(np.abs(np.asarray(s_gpu, dtype=np.float64) - s_ref).max()
+                               / max(np.abs(s_ref).max(), 1e-30)))
+        go, ro = np.concatenate(go), np.concatenate(ro)
+        eo = float(np.abs(go - ro).max() / max(np.abs(ro).max(), 1e-30))
+        bar = PARITY_BAR[dtype]
+        return {"o_max_rel_err": eo, "S_final_max_rel_err": es, "bar": bar,
+                "pass": bool(eo <= bar and es <= bar), "pairs": len(tasks),
+                "against": "fp64 oracle on the cpu_baseline sample"}
+    except Exception as e:  # noqa: BLE001 - reported in the line instead
+        return {"error": repr(e)[:300]}
+
+
+def cpu_baseline(inp, budget_s: float = 12.0, gpu_pair=None):
     """The fp64 oracle as it stands, on a bounded sample of (sequence, head)
-    pairs of the same workload, all host cores.  Tokens/s = token-heads / H / s."""
+    pairs of the same workload, all host cores.  Tokens/s = token-heads / H / s.
+    With ``gpu_pair`` the GPU's results for the sampled pairs are checked against
+    the oracle's (``parity``)."""
     import oracle
     cores = os.cpu_count() or 1
     cu = inp.offsets()
@@ -204,17 +233,23 @@ def cpu_baseline(inp, budget_s: float = 12.0):
     tasks = order[:n_pairs]
     threads = min(cores, n_pairs)
     t = time.perf_counter()
-    oracle.recurrent(inp.q, inp.k, inp.v, inp.log_alpha, inp.beta, inp.S0, cu, tasks=tasks,
-                     nthreads=threads)
+    outs, states = oracle.recurrent(inp.q, inp.k, inp.v, inp.log_alpha, inp.beta, inp.S0, cu,
+                                    tasks=tasks, nthreads=threads)
     dt = time.perf_counter() - t
     tok_heads = int(sum(lens[n] for n, _ in tasks))
-    return {"value": tok_heads / inp.H / dt, "unit": "tokens/s", "cores": threads,
-            "kind": "oracle", "seconds": round(dt, 3),
-            "sample": f"{n_pairs} of {inp.n_seqs * inp.H} (sequence, head) pairs, "
-                      f"{tok_heads} token-heads, fp64 recurrence, {threads} threads"}
+    res = {"value": tok_heads / inp.H / dt, "unit": "tokens/s", "cores": threads,
+           "kind": "oracle", "seconds": round(dt, 3),
+           "sample": f"{n_pairs} of {inp.n_seqs * inp.H} (sequence, head) pairs, "
+                     f"{tok_heads} token-heads, fp64 recurrence, {threads} threads"}
+    if gpu_pair is not None:
+        res["parity"] = sample_parity(tasks, outs, states, gpu_pair, inp.dtype)
+    return res
 
 
-def cpu_baseline_decode(ins, S0, budget_s: float = 12.0):
+def cpu_baseline_decode(ins, S0, budget_s: float = 12.0, gpu_pair=None):
+    """The fp64 oracle over the first steps of the decode workload from its initial state,
+    on a bounded sample of (sequence, head) states; ``gpu_pair`` as in cpu_baseline, the
+    GPU's o for those steps and its state after them."""
     import oracle
     cores = os.cpu_count() or 1
     N, H = ins[0].q.shape[0], ins[0].q.shape[1]
@@ -230,13 +265,16 @@ def cpu_baseline_decode(ins, S0, budget_s: float = 12.0):
     n_pairs = int(max(1, min(len(order), round(budget_s * cores / per_pair))))
     threads = min(cores, n_pairs)
     t = time.perf_counter()
-    oracle.recurrent(*arrs, S0, cu, tasks=order[:n_pairs], nthreads=threads)
+    outs, states = oracle.recurrent(*arrs, S0, cu, tasks=order[:n_pairs], nthreads=threads)
     dt = time.perf_counter() - t
     # a decode token is one sequence's step over all H heads
-    return {"value": n_pairs * steps / H / dt, "unit": "tokens/s", "cores": threads,
-            "kind": "oracle", "seconds": round(dt, 3),
-            "sample": f"{n_pairs} of {N * H} (sequence, head) states x {steps} steps, "
-                      f"fp64 recurrence, {threads} threads"}
+    res = {"value": n_pairs * steps / H / dt, "unit": "tokens/s", "cores": threads,
+           "kind": "oracle", "seconds": round(dt, 3),
+           "sample": f"{n_pairs} of {N * H} (sequence, head) states x {steps} steps, "
+                     f"fp64 recurrence, {threads} threads"}
+    if gpu_pair is not None:
+        res["parity"] = sample_parity(order[:n_pairs], outs, states, gpu_pair, ins[0].dtype)
+    return res
 
 
 # -------------------------------------------------------------------- the runs
@@ -364,11 +402,44 @@ def run_ours(args, rank, local_rank, world):
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         if name == "decode":
-            res["cpu_baseline"] = cpu_baseline_decode(ins[:min(4, len(ins))], S0,
-                                                      args.cpu_budget)
+            n_chk = min(4, len(ins))
+            try:
+                pairs = decode_pairs(dev_in[:n_chk], S0, device, kda_decode_step)
+            except Exception as e:  # noqa: BLE001 - reported by the parity entry instead
+                def pairs(n, hh, err=repr(e)):
+                    raise RuntimeError(err)
+            res["cpu_baseline"] = cpu_baseline_decode(ins[:n_chk], S0, args.cpu_budget, pairs)
         else:
-            res["cpu_baseline"] = cpu_baseline(inp_for_cpu, args.cpu_budget)
+            res["cpu_baseline"] = cpu_baseline(inp_for_cpu, args.cpu_budget, prefill_pairs(out, Sf, inp))
+        if "parity" in res["cpu_baseline"]:
+            res["parity"] = res["cpu_baseline"].pop("parity")
     return res
+
+
+def prefill_pairs(out, S_final, inp):
+    """gpu_pair(n, h) for a prefill call's results: o of sequence n's tokens at head h
+    (the token axis packed, whatever the view of ``out``) and its final state."""
+    o_flat, cu = out.view(-1, inp.H, inp.dv), inp.offsets()
+
+    def gpu_pair(n, hh):
+        o = o_flat[int(cu[n]):int(cu[n + 1]), hh].float().cpu().numpy()
+        return o, S_final[n, hh].cpu().numpy()
+    return gpu_pair
+
+
+def decode_pairs(dev_in, S0, device, kda_decode_step):
+    """The GPU's results for the decode steps the CPU baseline replays: the same step
+    inputs from the initial state, on a copy of it.  Returns gpu_pair(n, h)."""
+    import torch
+    S_chk = torch.from_numpy(S0).to(device, copy=True)
+    outs = [kda_decode_step(d["q"], d["k"], d["v"], d["log_alpha"], d["beta"], S_chk) for d in dev_in]
+    if torch.device(device).type == "cuda":
+        torch.cuda.synchronize(device)
+
+    def gpu_pair(n, hh):
+        o = torch.stack([o[n, hh] for o in outs]).float().cpu().numpy()
+        return o, S_chk[n, hh].cpu().numpy()
+    return gpu_pair
 
 
 def run_e2e(args, name, device, stream, rank):

@@ -54,3 +54,87 @@ def test_too_few_warmup_steps_are_refused(impl):
     r = run_bench(["--impl", impl, "--warmup", "2"])
     assert r.returncode != 0
     assert "--warmup must be >= 3" in r.stderr
+
+
+def test_sample_parity_reports_the_max_relative_error():
+    """The bench's parity check on the CPU-baseline sample: max|x - r| / max|r| over the
+    sampled pairs' o rows together and over each final state, and a failure to read the GPU
+    side reported in the line instead of raised."""
+    sys.path.insert(0, ROOT)
+    import numpy as np
+    import bench
+    rng = np.random.default_rng(5)
+    tasks = [(0, 0), (0, 1), (1, 0)]
+    outs = [rng.normal(size=(4, 3)) for _ in tasks]
+    states = [rng.normal(size=(2, 3)) for _ in tasks]
+    o_scale = max(np.abs(o).max() for o in outs)
+    perturbed = {t: (o + (0.5e-3 * o_scale if t == (0, 1) else 0.0), s * (1 + 1e-3))
+                 for t, o, s in zip(tasks, outs, states)}
+    p = bench.sample_parity(tasks, outs, states, lambda n, h: perturbed[(n, h)], "bf16")
+    assert abs(p["o_max_rel_err"] - 0.5e-3) < 1e-12
+    assert abs(p["S_final_max_rel_err"] - 1e-3) < 1e-12
+    assert p["pass"] is True and p["bar"] == 2e-2 and p["pairs"] == 3
+    assert bench.sample_parity(tasks, outs, states, lambda n, h: (outs[0] * 2, states[0]), "f32")["pass"] is False
+
+    def broken(n, h):
+        raise RuntimeError("no device")
+    assert "error" in bench.sample_parity(tasks, outs, states, broken, "bf16")
+
+
+def test_cpu_baseline_parity_of_the_oracle_against_itself_is_zero():
+    sys.path.insert(0, ROOT)
+    import numpy as np
+    import bench
+    import oracle
+    from gated_delta_rule_119_b200.inputs import make_inputs
+    oracle.build()
+    inp = make_inputs(2, 40, 2, 32, 32, "f32", 77, state=True, varlen=True)
+    cu = inp.offsets()
+    pairs = [(n, h) for n in range(inp.n_seqs) for h in range(inp.H)]
+    outs, states = oracle.recurrent(inp.q, inp.k, inp.v, inp.log_alpha, inp.beta, inp.S0, cu,
+                                    tasks=pairs)
+    ref = {t: (o, s) for t, o, s in zip(pairs, outs, states)}
+    cb = bench.cpu_baseline(inp, 0.2, lambda n, h: ref[(n, h)])
+    assert cb["parity"]["o_max_rel_err"] == 0.0 and cb["parity"]["S_final_max_rel_err"] == 0.0
+    assert cb["parity"]["pass"] is True and cb["kind"] == "oracle"
+
+
+def test_decode_parity_pairs_replay_the_steps_on_a_copy_of_the_state():
+    """decode_pairs runs the given decode steps from the initial state on a copy and returns,
+    per (sequence, head), the o of every step and the state after them (a stand-in step on
+    CPU tensors here: S += 1 per step, o = row sums of S)."""
+    sys.path.insert(0, ROOT)
+    import numpy as np
+    import torch
+    import bench
+
+    def fake_step(q, k, v, log_alpha, beta, S):
+        S += 1.0
+        return S.sum(dim=2)
+    S0 = np.arange(2 * 3 * 4 * 5, dtype=np.float32).reshape(2, 3, 4, 5)
+    dev_in = [dict(q=None, k=None, v=None, log_alpha=None, beta=None) for _ in range(3)]
+    pair = bench.decode_pairs(dev_in, S0, torch.device("cpu"), fake_step)
+    o, S = pair(1, 2)
+    assert o.shape == (3, 5) and S.shape == (4, 5)
+    np.testing.assert_allclose(S, S0[1, 2] + 3)
+    np.testing.assert_allclose(o[0], (S0[1, 2] + 1).sum(0))
+    assert S0[1, 2, 0, 0] == 1 * 60 + 2 * 20          # the initial state is untouched
+
+
+def test_prefill_parity_pairs_index_the_packed_token_axis():
+    sys.path.insert(0, ROOT)
+    import numpy as np
+    import torch
+    import bench
+    from gated_delta_rule_119_b200.inputs import make_inputs
+    inp = make_inputs(3, 50, 2, 32, 32, "f32", 78, varlen=True)
+    cu = inp.offsets()
+    out = torch.arange(inp.total_tokens * 2 * 32, dtype=torch.float32).view(inp.total_tokens, 2, 32)
+    Sf = torch.randn(3, 2, 32, 32)
+    o, S = bench.prefill_pairs(out, Sf, inp)(2, 1)
+    np.testing.assert_array_equal(o, out[cu[2]:cu[3], 1].numpy())
+    np.testing.assert_array_equal(S, Sf[2, 1].numpy())
+    fixed = make_inputs(2, 7, 3, 32, 32, "f32", 79)
+    out4 = torch.randn(2, 7, 3, 32)                    # the [B, T, H, dv] view of a fixed-length call
+    o, _ = bench.prefill_pairs(out4, torch.zeros(2, 3, 32, 32), fixed)(1, 2)
+    np.testing.assert_array_equal(o, out4[1, :, 2].numpy())
