@@ -187,26 +187,34 @@ def measured_peaks():
 PARITY_BAR = {"bf16": 2e-2, "f32": 1e-4}
 
 
+def _rel(x, r) -> float:
+    x, r = np.asarray(x, dtype=np.float64), np.asarray(r, dtype=np.float64)
+    return float(np.abs(x - r).max() / max(np.abs(r).max(), 1e-30))
+
+
 def sample_parity(tasks, outs, states, gpu_pair, dtype: str) -> dict:
-    """Max relative error, max|x - r| / max|r|, of the GPU's o (over the sampled pairs' rows
-    together) and of each final state, against the oracle's results for the same (sequence,
-    head) pairs.  gpu_pair(n, h) -> (o [len, dv], S [dk, dv]).  A failure to read the GPU's
-    result is reported in place of the numbers; it never stops the bench."""
+    """Max relative error, max|x - r| / max|r|, of the GPU's o and final states against the
+    oracle's results for the same (sequence, head) pairs, pooled over the pairs and for the
+    worst pair on its own.  gpu_pair(n, h) -> (o [len, dv], S [dk, dv]).  A failure to read
+    the GPU's result is reported in place of the numbers; it never stops the bench."""
     try:
-        go, ro, es = [], [], 0.0
+        go, ro, gs, rs, po, ps = [], [], [], [], [], []
         for (n, h), o_ref, s_ref in zip(tasks, outs, states):
             o_gpu, s_gpu = gpu_pair(n, h)
-            go.append(np.asarray(o_gpu, dtype=np.float64).ravel())
-            ro.append(np.asarray(o_ref, dtype=np.float64).ravel())
-            s_ref = np.asarray(s_ref, dtype=np.float64)
-            es = max(es, float(np.abs(np.asarray(s_gpu, dtype=np.float64) - s_ref).max()
-                               / max(np.abs(s_ref).max(), 1e-30)))
-        go, ro = np.concatenate(go), np.concatenate(ro)
-        eo = float(np.abs(go - ro).max() / max(np.abs(ro).max(), 1e-30))
+            if np.size(o_ref):
+                go.append(np.asarray(o_gpu, dtype=np.float64).ravel())
+                ro.append(np.asarray(o_ref, dtype=np.float64).ravel())
+                po.append(_rel(o_gpu, o_ref))
+            gs.append(np.asarray(s_gpu, dtype=np.float64).ravel())
+            rs.append(np.asarray(s_ref, dtype=np.float64).ravel())
+            ps.append(_rel(s_gpu, s_ref))
+        eo = _rel(np.concatenate(go), np.concatenate(ro))
+        es = _rel(np.concatenate(gs), np.concatenate(rs))
         bar = PARITY_BAR[dtype]
-        return {"o_max_rel_err": eo, "S_final_max_rel_err": es, "bar": bar,
-                "pass": bool(eo <= bar and es <= bar), "pairs": len(tasks),
-                "against": "fp64 oracle on the cpu_baseline sample"}
+        return {"o_max_rel_err": eo, "S_final_max_rel_err": es,
+                "o_worst_pair_rel_err": max(po), "S_final_worst_pair_rel_err": max(ps),
+                "bar": bar, "pass": bool(max(eo, es, max(po), max(ps)) <= bar),
+                "pairs": len(tasks), "against": "fp64 oracle, same (sequence, head) pairs"}
     except Exception as e:  # noqa: BLE001 - reported in the line instead
         return {"error": repr(e)[:300]}
 
@@ -288,19 +296,15 @@ def workload_config(name, inp_or_dims, n_gpus):
     return cfg
 
 
-def run_ours(args, rank, local_rank, world):
+def setup_workload(name, args, device, rank):
+    """Inputs of one workload resident on the device and the step that runs it.  Returns a
+    dict: step(i), units per step (tokens), algorithmic bytes and FLOPs per step, the
+    kernel key, kernel launches per step, and parity(budget_s) -> the oracle's CPU baseline
+    on a bounded sample with the GPU's results for the same pairs checked against it."""
     import torch
-    from gated_delta_rule_119_b200 import kda_chunk_fwd, kda_decode_step, load_library
-    load_library()
-    device = torch.device("cuda", local_rank)
-    torch.cuda.set_device(device)
-    name = args.workload
+    from gated_delta_rule_119_b200 import kda_chunk_fwd, kda_decode_step
     w = WORKLOADS[name]
-    hbm, bf16_tf, peak_kind = measured_peaks()
-    stream = torch.cuda.current_stream(device)
     es = 2 if w["dtype"] == "bf16" else 4
-    launches_per_step = 1        # decode: one kernel; SIMT prefill: one kernel
-
     if name == "decode":
         N, H, dk, dv = w["B"], w["H"], w["dk"], w["dv"]
         n_in = max(1, min(args.decode_inputs, args.steps + args.warmup))
@@ -314,106 +318,194 @@ def run_ours(args, rank, local_rank, world):
         def step(i):
             d = dev_in[i % n_in]
             kda_decode_step(d["q"], d["k"], d["v"], d["log_alpha"], d["beta"], S, out)
-        units_per_step = N                       # tokens (one per sequence)
-        bytes_per_launch = alg_bytes_decode(N * H, dk, dv, es)
-        flops_per_launch = N * H * 7 * dk * dv
-        kernel_key = "decode"
-        inp_for_cpu = None
-    else:
-        inp = make_workload(name) if rank == 0 else make_inputs(
-            w["B"], w["T"], w["H"], w["dk"], w["dv"], w["dtype"], rank_seed(w["index"], rank),
-            state=w["state"], varlen=w["varlen"], gates=w["gates"])
-        d = to_torch(inp, device)
-        out = torch.empty(d["v"].shape, dtype=d["q"].dtype, device=device)
-        Sf = torch.empty((inp.n_seqs, inp.H, inp.dk, inp.dv), dtype=torch.float32, device=device)
 
-        def step(i):
-            kda_chunk_fwd(d["q"], d["k"], d["v"], d["log_alpha"], d["beta"], d["S0"],
-                          d["cu_seqlens"], out, Sf)
-        tok_heads = inp.total_tokens * inp.H
-        units_per_step = inp.total_tokens
-        bytes_per_launch = alg_bytes_prefill(tok_heads, inp.n_seqs * inp.H, inp.dk, inp.dv, es,
-                                             inp.S0 is not None, True)
-        flops_per_launch = alg_flops_prefill(tok_heads, inp.dk, inp.dv)
-        kernel_key = "chunk" if (w["dtype"] == "bf16" and w["dk"] == 128 and w["dv"] == 128) \
-            else "chunk_simt"
-        if kernel_key == "chunk":
-            # intra-chunk kernel + scan kernel, plus the slot-offset kernel for varlen
-            launches_per_step = 2 + (inp.cu_seqlens is not None)
-        inp_for_cpu = inp
-
-    for i in range(args.warmup):
-        step(i)
-    torch.cuda.synchronize(device)
-    barrier(device)
-    torch.cuda.synchronize(device)
-    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    with ClockSampler(device.index if device.index is not None else 0) as clk:
-        ev0.record(stream)
-        for i in range(args.steps):
-            step(args.warmup + i)
-        ev1.record(stream)
-        torch.cuda.synchronize(device)
-    barrier(device)
-    torch.cuda.synchronize(device)
-    ms_local = ev0.elapsed_time(ev1) / args.steps
-    ms = reduce_max(ms_local, device)
-
-    # Duration of one call, events around each call on the launching stream.  For the
-    # tensor-core prefill a call is its two kernels back to back (intra-chunk, then
-    # scan); the roofline is taken over the call because the algorithmic bytes (q, k,
-    # v, gates in; o and states out) belong to the pair, not to either kernel alone.
-    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-           for _ in range(min(args.steps, 20))]
-    for i, (a, b) in enumerate(evs):
-        a.record(stream)
-        step(i)
-        b.record(stream)
-    torch.cuda.synchronize(device)
-    launch_ms = float(np.mean([a.elapsed_time(b) for a, b in evs]))
-    launch_ms = reduce_max(launch_ms, device)
-
-    # end to end through the public API with host buffers
-    e2e = run_e2e(args, name, device, stream, rank)
-
-    value = units_per_step * world / (ms / 1e3)
-    achieved = bytes_per_launch / (launch_ms / 1e3) / 1e9
-    traffic = profiled_traffic(kernel_key, name)
-    res = {
-        "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
-        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
-        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
-        "dtype": w["dtype"], "data": "synthetic (seeded numpy; see inputs.py recipe)",
-        "config": {**workload_config(name, None, world),
-                   "l2": "no flush: the inputs of one step exceed the 126 MB L2"
-                   if bytes_per_launch > 126e6 else "inputs fit in L2; reported as is"},
-        "tflops": flops_per_launch / (launch_ms / 1e3) / 1e12,
-        "roofline": {"bound": "hbm", "achieved": achieved, "peak": hbm, "unit": "GB/s",
-                     "frac": achieved / hbm, "traffic": traffic,
-                     "peak_kind": f"{peak_kind} (STREAM-style copy, burst)",
-                     "kernel": {"chunk": "kda_chunk_intra_kernel + kda_chunk_scan_kernel "
-                                          "(one kda_chunk_fwd call)",
-                                "chunk_simt": "kda_chunk_simt_kernel",
-                                "decode": "kda_decode_kernel"}[kernel_key],
-                     "alg_bytes_per_launch": bytes_per_launch, "launch_ms": launch_ms},
-        "clocks": clk.summary(),
-        "e2e": e2e,
-        "gpu_launches": args.steps * launches_per_step,
-    }
-    if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        if name == "decode":
+        def parity(budget):
             n_chk = min(4, len(ins))
             try:
                 pairs = decode_pairs(dev_in[:n_chk], S0, device, kda_decode_step)
             except Exception as e:  # noqa: BLE001 - reported by the parity entry instead
                 def pairs(n, hh, err=repr(e)):
                     raise RuntimeError(err)
-            res["cpu_baseline"] = cpu_baseline_decode(ins[:n_chk], S0, args.cpu_budget, pairs)
-        else:
-            res["cpu_baseline"] = cpu_baseline(inp_for_cpu, args.cpu_budget, prefill_pairs(out, Sf, inp))
+            return cpu_baseline_decode(ins[:n_chk], S0, budget, pairs)
+        return dict(step=step, units=N, bytes=alg_bytes_decode(N * H, dk, dv, es),
+                    flops=N * H * 7 * dk * dv, kernel_key="decode", launches=1, parity=parity,
+                    hold=(dev_in, S, out))
+    inp = make_workload(name) if rank == 0 else make_inputs(
+        w["B"], w["T"], w["H"], w["dk"], w["dv"], w["dtype"], rank_seed(w["index"], rank),
+        state=w["state"], varlen=w["varlen"], gates=w["gates"])
+    d = to_torch(inp, device)
+    out = torch.empty(d["v"].shape, dtype=d["q"].dtype, device=device)
+    Sf = torch.empty((inp.n_seqs, inp.H, inp.dk, inp.dv), dtype=torch.float32, device=device)
+
+    def step(i):
+        kda_chunk_fwd(d["q"], d["k"], d["v"], d["log_alpha"], d["beta"], d["S0"],
+                      d["cu_seqlens"], out, Sf)
+
+    def parity(budget):
+        return cpu_baseline(inp, budget, prefill_pairs(out, Sf, inp))
+    tok_heads = inp.total_tokens * inp.H
+    tc = w["dtype"] == "bf16" and w["dk"] == 128 and w["dv"] == 128
+    return dict(step=step, units=inp.total_tokens,
+                bytes=alg_bytes_prefill(tok_heads, inp.n_seqs * inp.H, inp.dk, inp.dv, es,
+                                        inp.S0 is not None, True),
+                flops=alg_flops_prefill(tok_heads, inp.dk, inp.dv),
+                kernel_key="chunk" if tc else "chunk_simt",
+                # intra-chunk kernel + scan kernel, plus the slot-offset kernel for varlen
+                launches=(2 + (inp.cu_seqlens is not None)) if tc else 1,
+                parity=parity, hold=(d, out, Sf))
+
+
+def time_steps(step, steps, warmup, device, stream, min_timed_s=1.0, min_passes=5,
+               max_passes=200, sampler=None):
+    """W untimed warm-up steps, then passes of exactly `steps` timed steps, each pass
+    bracketed by CUDA events on the launching stream with a synchronize after it; at least
+    `min_passes` passes and until about `min_timed_s` of timed work.  A barrier and a device
+    synchronize stand on both sides of the timed region.  Returns ms per step of each pass."""
+    import torch
+    for i in range(warmup):
+        step(i)
+    torch.cuda.synchronize(device)
+    barrier(device)
+    torch.cuda.synchronize(device)
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    passes = []
+    with (sampler if sampler is not None else _NullCtx()):
+        while True:
+            ev0.record(stream)
+            for i in range(steps):
+                step(warmup + i)
+            ev1.record(stream)
+            torch.cuda.synchronize(device)
+            passes.append(ev0.elapsed_time(ev1) / steps)
+            done_s = sum(passes) * steps / 1e3
+            if len(passes) >= max_passes or (len(passes) >= min_passes and done_s >= min_timed_s):
+                break
+    barrier(device)
+    torch.cuda.synchronize(device)
+    return passes
+
+
+class _NullCtx:
+    def __enter__(self):
+        return self
+
+    def __exit__(self, *exc):
+        return False
+
+
+def launch_duration_ms(step, n, device, stream):
+    """Mean duration of one call, CUDA events around each call on the launching stream.
+    For the tensor-core prefill a call is its kernels back to back (intra-chunk, then
+    scan); the roofline is taken over the call because the algorithmic bytes (q, k, v,
+    gates in; o and states out) belong to the pair, not to either kernel alone."""
+    import torch
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+           for _ in range(n)]
+    for i, (a, b) in enumerate(evs):
+        a.record(stream)
+        step(i)
+        b.record(stream)
+    torch.cuda.synchronize(device)
+    return float(np.mean([a.elapsed_time(b) for a, b in evs]))
+
+
+def roofline_entry(wl, launch_ms, hbm, peak_kind, name):
+    achieved = wl["bytes"] / (launch_ms / 1e3) / 1e9
+    return {"bound": "hbm", "achieved": achieved, "peak": hbm, "unit": "GB/s",
+            "frac": achieved / hbm, "traffic": profiled_traffic(wl["kernel_key"], name),
+            "peak_kind": f"{peak_kind} (STREAM-style copy, burst)",
+            "kernel": {"chunk": "kda_chunk_intra_kernel + kda_chunk_scan_kernel "
+                                "(one kda_chunk_fwd call)",
+                       "chunk_simt": "kda_chunk_simt_kernel",
+                       "decode": "kda_decode_kernel"}[wl["kernel_key"]],
+            "alg_bytes_per_launch": wl["bytes"], "launch_ms": launch_ms}
+
+
+def run_ours(args, rank, local_rank, world):
+    import torch
+    from gated_delta_rule_119_b200 import load_library
+    load_library()
+    device = torch.device("cuda", local_rank)
+    torch.cuda.set_device(device)
+    name = args.workload
+    w = WORKLOADS[name]
+    hbm, bf16_tf, peak_kind = measured_peaks()
+    stream = torch.cuda.current_stream(device)
+    wl = setup_workload(name, args, device, rank)
+
+    clk = ClockSampler(device.index if device.index is not None else 0)
+    passes = time_steps(wl["step"], args.steps, args.warmup, device, stream,
+                        min_timed_s=args.min_timed_s, sampler=clk)
+    ms = reduce_max(statistics.median(passes), device)
+    launch_ms = reduce_max(launch_duration_ms(wl["step"], min(args.steps, 20), device, stream),
+                           device)
+
+    # end to end through the public API with host buffers
+    e2e = run_e2e(args, name, device, stream, rank)
+
+    value = wl["units"] * world / (ms / 1e3)
+    res = {
+        "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
+        "timed_passes": {"passes": len(passes), "median_ms": statistics.median(passes),
+                         "min_ms": min(passes), "max_ms": max(passes),
+                         "note": f"each pass times exactly {args.steps} steps; ms_per_step is "
+                                 "the median pass (max over ranks)"},
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": w["dtype"], "data": "synthetic (seeded numpy; see inputs.py recipe)",
+        "config": {**workload_config(name, None, world),
+                   "l2": "no flush: the inputs of one step exceed the 126 MB L2"
+                   if wl["bytes"] > 126e6 else "inputs fit in L2; reported as is"},
+        "tflops": wl["flops"] / (launch_ms / 1e3) / 1e12,
+        "roofline": roofline_entry(wl, launch_ms, hbm, peak_kind, name),
+        "clocks": clk.summary(),
+        "e2e": e2e,
+        "gpu_launches": args.steps * len(passes) * wl["launches"],
+        "gpu_launches_note": "kernel launches of this library inside the timed region "
+                             f"({wl['launches']} per step, {len(passes)} passes of "
+                             f"{args.steps} steps)",
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        res["cpu_baseline"] = wl["parity"](args.cpu_budget)
         if "parity" in res["cpu_baseline"]:
             res["parity"] = res["cpu_baseline"].pop("parity")
+    del wl
+    torch.cuda.empty_cache()
+    if world == 1 and args.workloads:
+        res["workloads"] = {}
+        for other in [x for x in args.workloads.split(",") if x and x != name]:
+            res["workloads"][other] = run_other_workload(other, args, device, stream, rank,
+                                                         hbm, peak_kind)
+            torch.cuda.empty_cache()
     return res
+
+
+def run_other_workload(name, args, device, stream, rank, hbm, peak_kind):
+    """One more workload in the same process: ms per step (median of timed passes), tokens/s,
+    its roofline and parity on a bounded oracle sample.  Failures are reported, not raised."""
+    try:
+        wl = setup_workload(name, args, device, rank)
+        steps = min(args.steps, 20)
+        clk = ClockSampler(device.index if device.index is not None else 0)
+        passes = time_steps(wl["step"], steps, 3, device, stream, min_timed_s=0.3, sampler=clk)
+        launch_ms = launch_duration_ms(wl["step"], min(steps, 10), device, stream)
+        ms = statistics.median(passes)
+        w = WORKLOADS[name]
+        entry = {"ms_per_step": ms, "min_ms": min(passes), "max_ms": max(passes),
+                 "passes": len(passes), "steps_per_pass": steps,
+                 "value": wl["units"] / (ms / 1e3), "unit": "tokens/s",
+                 "tflops": wl["flops"] / (launch_ms / 1e3) / 1e12,
+                 "roofline": roofline_entry(wl, launch_ms, hbm, peak_kind, name),
+                 "clocks": clk.summary(), "gpu_launches_per_step": wl["launches"],
+                 "config": workload_config(name, None, 1)}
+        if not args.no_cpu_baseline:
+            cb = wl["parity"](args.workload_parity_budget)
+            entry["parity"] = cb.pop("parity", None)
+            entry["cpu_baseline"] = cb
+        del wl
+        return entry
+    except Exception as e:  # noqa: BLE001 - reported in the line instead
+        return {"error": repr(e)[:300], "dtype": WORKLOADS[name]["dtype"]}
 
 
 def prefill_pairs(out, S_final, inp):
@@ -546,6 +638,13 @@ def main(argv=None):
                     help="seconds of host-core work for the CPU baseline sample")
     ap.add_argument("--ref-step-budget", type=float, default=4.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--min-timed-s", type=float, default=1.0,
+                    help="repeat the timed passes of --steps steps until about this much "
+                         "timed work (at least 5 passes)")
+    ap.add_argument("--workloads", default="decode,varlen,extremes",
+                    help="other workloads measured in the same process at N=1 (comma list; "
+                         "empty for none)")
+    ap.add_argument("--workload-parity-budget", type=float, default=3.0)
     args = ap.parse_args(argv)
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")

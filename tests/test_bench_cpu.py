@@ -58,7 +58,7 @@ def test_too_few_warmup_steps_are_refused(impl):
 
 def test_sample_parity_reports_the_max_relative_error():
     """The bench's parity check on the CPU-baseline sample: max|x - r| / max|r| over the
-    sampled pairs' o rows together and over each final state, and a failure to read the GPU
+    sampled pairs together and for the worst pair on its own, and a failure to read the GPU
     side reported in the line instead of raised."""
     sys.path.insert(0, ROOT)
     import numpy as np
@@ -66,6 +66,7 @@ def test_sample_parity_reports_the_max_relative_error():
     rng = np.random.default_rng(5)
     tasks = [(0, 0), (0, 1), (1, 0)]
     outs = [rng.normal(size=(4, 3)) for _ in tasks]
+    outs[1] *= 0.1                                   # a pair with small outputs of its own
     states = [rng.normal(size=(2, 3)) for _ in tasks]
     o_scale = max(np.abs(o).max() for o in outs)
     perturbed = {t: (o + (0.5e-3 * o_scale if t == (0, 1) else 0.0), s * (1 + 1e-3))
@@ -73,6 +74,10 @@ def test_sample_parity_reports_the_max_relative_error():
     p = bench.sample_parity(tasks, outs, states, lambda n, h: perturbed[(n, h)], "bf16")
     assert abs(p["o_max_rel_err"] - 0.5e-3) < 1e-12
     assert abs(p["S_final_max_rel_err"] - 1e-3) < 1e-12
+    # the worst pair on its own: pair (0, 1)'s shift relative to its own largest |o|
+    assert abs(p["o_worst_pair_rel_err"] - 0.5e-3 * o_scale / np.abs(outs[1]).max()) < 1e-12
+    assert p["o_worst_pair_rel_err"] > p["o_max_rel_err"]
+    assert abs(p["S_final_worst_pair_rel_err"] - 1e-3) < 1e-12
     assert p["pass"] is True and p["bar"] == 2e-2 and p["pairs"] == 3
     assert bench.sample_parity(tasks, outs, states, lambda n, h: (outs[0] * 2, states[0]), "f32")["pass"] is False
 
