@@ -35,14 +35,15 @@ ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
 from gated_delta_rule_119_b200.inputs import (WORKLOADS, make_decode_state,  # noqa: E402
-                                             make_decode_step, make_inputs, make_workload,
-                                             to_torch)
+                                             make_decode_step, make_form_inputs, make_inputs,
+                                             make_workload, to_torch)
 
 METRIC = ("KDA prefill tokens/s + TFLOP/s (% roofline) at dk=dv=128; "
           "decode tokens/s, % HBM BW")
 PROFILES = os.path.join(ROOT, "profiles")
 KERNEL_SOURCES = {"chunk": "gated_delta_rule_119_b200/csrc/kda_chunk_tc.cu",
                   "chunk_simt": "gated_delta_rule_119_b200/csrc/kda_chunk_simt.cuh",
+                  "chunk_bwd": "gated_delta_rule_119_b200/csrc/kda_chunk_bwd.cu",
                   "decode": "gated_delta_rule_119_b200/csrc/kda_decode.cu"}
 
 
@@ -61,8 +62,39 @@ def alg_flops_prefill(n_tok_heads: int, dk: int, dv: int, C: int = 64) -> int:
     return n_tok_heads * (6 * dk * dv + 2 * C * (dk + dv) + C * C // 3)
 
 
-def alg_bytes_decode(n_pairs: int, dk: int, dv: int, es: int) -> int:
-    return n_pairs * (2 * dk * dv * 4 + es * (2 * dk + 2 * dv) + 4 * dk + 4)
+def alg_bytes_decode(n_pairs: int, dk: int, dv: int, es: int, L: int = 1) -> int:
+    """Per (sequence, head): the fp32 state read once and written once, and for each of the
+    L tokens q, k, v, o in the input dtype, log_alpha and beta fp32."""
+    return n_pairs * (2 * dk * dv * 4 + L * (es * (2 * dk + 2 * dv) + 4 * dk + 4))
+
+
+def gate_bytes_per_token_head(form: str, dk: int, es: int) -> int:
+    """The gate stream of one token-head: per-channel log_alpha fp32, one fp32 scalar, none,
+    or the fused gate's f in the input dtype."""
+    return {"channel": 4 * dk, "scalar": 4, "none": 0, "fused": es * dk}[form]
+
+
+# Variants of the workloads for the extended entry points, measured in the workloads object:
+# (base workload, gate form, unnormalised q/k + beta logits, decode tokens per call, indexed pool).
+# The fused gate's parameters are A_log = dt_bias = 0 here, so its decay has the default gates'
+# distribution and the comparison with "prefill" isolates the cost of the in-kernel front-end.
+VARIANTS = {
+    "prefill_fused": ("prefill", "fused", True, 1, False),
+    "prefill_gdn": ("prefill", "scalar", False, 1, False),
+    "prefill_bwd": ("prefill", "channel", False, 1, False),
+    "decode_indexed": ("decode", "channel", False, 1, True),
+    "decode_mtp4": ("decode", "channel", False, 4, True),
+}
+# fp32 FMA peak of the B200 from its unit counts: 148 SMs x 128 fp32 lanes x 2 flops x 1.965 GHz
+FP32_PEAK_TFLOPS = 148 * 128 * 2 * 1.965e9 / 1e12
+
+
+def alg_flops_backward(n_tok_heads: int, dk: int, dv: int, C: int = 16) -> int:
+    """The backward's state-sized products per token-head, forward recomputation included:
+    r = v - (k gamma) S and the state update (4 dk dv), du's (k kappa) dS' (2 dk dv), the previous
+    chunk's dS (4 dk dv), d(s q gamma), d(k gamma), d(k kappa) (6 dk dv) and d gamma_last (dk dv);
+    plus the C x C products of the chunk (8 C (dk + dv))."""
+    return n_tok_heads * (17 * dk * dv + 8 * C * (dk + dv))
 
 
 # ----------------------------------------------------------- distributed plumbing
@@ -254,6 +286,110 @@ def cpu_baseline(inp, budget_s: float = 12.0, gpu_pair=None):
     return res
 
 
+def oracle_view(inp):
+    """The batch as the oracle reads it for a gate form of the extended entry points: the
+    oracle's own gate front-end (oracle/gates.py) applied to the bytes the GPU receives --
+    per-channel log alpha, beta after the sigmoid, unit-length q and k where the flags ask."""
+    import dataclasses
+    from oracle import gates
+    q, k, beta = inp.q, inp.k, inp.beta
+    if inp.form == "scalar":
+        la = gates.broadcast_scalar(inp.log_alpha, inp.dk)
+    elif inp.form == "none":
+        la = np.zeros(inp.q.shape)
+    elif inp.form == "fused":
+        la = gates.fused_log_alpha(inp.f, inp.A_log, inp.dt_bias)
+    else:
+        la = inp.log_alpha
+    if inp.flags & 1:
+        q = gates.l2_normalize(q)
+    if inp.flags & 2:
+        k = gates.l2_normalize(k)
+    if inp.flags & 4:
+        beta = gates.sigmoid(beta)
+    return dataclasses.replace(inp, q=q, k=k, log_alpha=la, beta=beta)
+
+
+def cpu_baseline_backward(inp, dO, dSf, holder, budget_s):
+    """The fp64 reverse-mode oracle on a bounded sample of (sequence, head) pairs of a backward
+    workload; parity of every gradient of the GPU's last call (holder["g"]) against it, the
+    worst over the gradients and pairs."""
+    import oracle
+    import torch
+    cores = os.cpu_count() or 1
+    cu = inp.offsets()
+    lens = np.diff(cu)
+    order = [(n, h) for n in range(inp.n_seqs) for h in range(inp.H) if lens[n] > 0]
+    t = time.perf_counter()
+    oracle.backward(inp.q, inp.k, inp.v, inp.log_alpha, inp.beta, inp.S0, cu, dO, dSf,
+                    tasks=order[:1], nthreads=1)
+    per_pair = max(time.perf_counter() - t, 1e-6)
+    n_pairs = int(max(1, min(len(order), round(budget_s * cores / per_pair))))
+    threads = min(cores, n_pairs)
+    t = time.perf_counter()
+    r = oracle.backward(inp.q, inp.k, inp.v, inp.log_alpha, inp.beta, inp.S0, cu, dO, dSf,
+                        tasks=order[:n_pairs], nthreads=threads)
+    dt = time.perf_counter() - t
+    res = {"value": sum(int(lens[n]) for n, _ in order[:n_pairs]) / inp.H / dt, "unit": "tokens/s",
+           "cores": threads, "kind": "oracle", "seconds": round(dt, 3),
+           "sample": f"{n_pairs} of {inp.n_seqs * inp.H} (sequence, head) pairs, fp64 reverse mode, "
+                     f"{threads} threads"}
+    try:
+        g = holder["g"]
+        torch.cuda.synchronize()
+        T, H = inp.total_tokens, inp.H
+        gpu = {"dq": g["dq"].float().cpu().numpy().reshape(T, H, -1),
+               "dk": g["dk"].float().cpu().numpy().reshape(T, H, -1),
+               "dv": g["dv"].float().cpu().numpy().reshape(T, H, -1),
+               "dlog_alpha": g["dgate"].cpu().numpy().reshape(T, H, -1),
+               "dbeta": g["dbeta"].cpu().numpy().reshape(T, H), "dS0": g["dS0"].cpu().numpy()}
+        worst, bar = {}, PARITY_BAR[inp.dtype]
+        for name, ref in r.items():
+            errs = []
+            for n, h in order[:n_pairs]:
+                x = gpu[name][n, h] if name == "dS0" else gpu[name][cu[n]:cu[n + 1], h]
+                y = ref[n, h] if name == "dS0" else ref[cu[n]:cu[n + 1], h]
+                errs.append(_rel(x, y))
+            worst[name] = max(errs)
+        res["parity"] = {"worst_pair_rel_err": worst, "bar": bar, "pass": bool(max(worst.values()) <= bar),
+                         "pairs": n_pairs, "against": "fp64 reverse-mode oracle, same pairs"}
+    except Exception as e:  # noqa: BLE001 - reported in the line instead
+        res["parity"] = {"error": repr(e)[:300]}
+    return res
+
+
+def cpu_baseline_decode_ex(ins, S0, L, budget_s, gpu_pair):
+    """The oracle over the first calls of a decode variant (L tokens per sequence per call,
+    ins[j] packed sequence-major [N * L, H, .]) from each sequence's initial state S0 [N, H,
+    dk, dv], on a bounded sample of (sequence, head) pairs; parity against gpu_pair."""
+    import oracle
+    cores = os.cpu_count() or 1
+    views = [oracle_view(i) for i in ins]
+    N, H = ins[0].n_seqs, ins[0].H
+    calls = len(views)
+
+    def stack(name):
+        xs = [np.asarray(getattr(v, name)) for v in views]
+        return np.stack([x.reshape(N, L, *x.shape[1:]) for x in xs], 1).reshape(N * calls * L, *xs[0].shape[1:])
+    arrs = [stack(x) for x in ("q", "k", "v", "log_alpha", "beta")]
+    cu = np.arange(N + 1) * calls * L
+    order = [(n, h) for n in range(N) for h in range(H)]
+    t = time.perf_counter()
+    oracle.recurrent(*arrs, S0, cu, tasks=order[:1], nthreads=1)
+    per_pair = max(time.perf_counter() - t, 1e-6)
+    n_pairs = int(max(1, min(len(order), round(budget_s * cores / per_pair))))
+    threads = min(cores, n_pairs)
+    t = time.perf_counter()
+    outs, states = oracle.recurrent(*arrs, S0, cu, tasks=order[:n_pairs], nthreads=threads)
+    dt = time.perf_counter() - t
+    res = {"value": n_pairs * calls * L / H / dt, "unit": "tokens/s", "cores": threads, "kind": "oracle",
+           "seconds": round(dt, 3),
+           "sample": f"{n_pairs} of {N * H} (sequence, head) states x {calls} calls of {L} tokens, "
+                     f"fp64 recurrence, {threads} threads"}
+    res["parity"] = sample_parity(order[:n_pairs], outs, states, gpu_pair, ins[0].dtype)
+    return res
+
+
 def cpu_baseline_decode(ins, S0, budget_s: float = 12.0, gpu_pair=None):
     """The fp64 oracle over the first steps of the decode workload from its initial state,
     on a bounded sample of (sequence, head) states; ``gpu_pair`` as in cpu_baseline, the
@@ -303,6 +439,8 @@ def setup_workload(name, args, device, rank):
     on a bounded sample with the GPU's results for the same pairs checked against it."""
     import torch
     from gated_delta_rule_119_b200 import kda_chunk_fwd, kda_decode_step
+    if name in VARIANTS:
+        return setup_variant(name, args, device, rank)
     w = WORKLOADS[name]
     es = 2 if w["dtype"] == "bf16" else 4
     if name == "decode":
@@ -353,6 +491,110 @@ def setup_workload(name, args, device, rank):
                 # intra-chunk kernel + scan kernel, plus the slot-offset kernel for varlen
                 launches=(2 + (inp.cu_seqlens is not None)) if tc else 1,
                 parity=parity, hold=(d, out, Sf))
+
+
+def setup_variant(name, args, device, rank):
+    """A VARIANTS entry: the base workload's shapes through kda_chunk_fwd_ex / kda_decode_ex,
+    in the same dict form as setup_workload."""
+    import torch
+    from gated_delta_rule_119_b200 import kda_chunk_fwd_ex, kda_decode_ex
+    base, form, raw, L, indexed = VARIANTS[name]
+    w = WORKLOADS[base]
+    es = 2 if w["dtype"] == "bf16" else 4
+    kind = {"channel": 0, "scalar": 1, "none": 2, "fused": 3}[form]
+    flags = dict(norm_q=raw, norm_k=raw, beta_logits=raw)
+    if base == "decode":
+        N, H, dk, dv = w["B"], w["H"], w["dk"], w["dv"]
+        n_in = max(1, min(args.decode_inputs // L, args.steps + args.warmup))
+        ins = [make_form_inputs(N, L, H, dk, dv, w["dtype"], (rank_seed(w["index"], rank), t), form,
+                                raw=raw) for t in range(n_in)]
+        pool0 = make_decode_state(N, H, dk, dv, rank_seed(w["index"], rank))
+        perm = np.random.default_rng(11).permutation(N).astype(np.int32) if indexed else None
+        dev_in = [to_torch(i, device) for i in ins]
+        pool = torch.from_numpy(pool0).to(device)
+        idx = torch.from_numpy(perm).to(device) if indexed else None
+        out = torch.empty((N, L, H, dv), dtype=dev_in[0]["q"].dtype, device=device)
+
+        def call(d, pool_, out_):
+            gate = d["f"] if form == "fused" else d["log_alpha"]
+            kda_decode_ex(d["q"], d["k"], d["v"], gate, d["beta"], pool_, idx, out_, gate_kind=kind,
+                          A_log=d["A_log"], dt_bias=d["dt_bias"], **flags)
+
+        def step(i):
+            call(dev_in[i % n_in], pool, out)
+
+        def parity(budget):
+            n_chk = min(2, n_in)
+            chk = torch.from_numpy(pool0).to(device)
+            outs = []
+            for d in dev_in[:n_chk]:
+                o_ = torch.empty_like(out)
+                call(d, chk, o_)
+                outs.append(o_)
+            torch.cuda.synchronize(device)
+            slot = perm if indexed else np.arange(N)
+
+            def gpu_pair(n, hh):
+                o = torch.cat([o_[n, :, hh] for o_ in outs]).float().cpu().numpy()
+                return o, chk[int(slot[n]), hh].cpu().numpy()
+            return cpu_baseline_decode_ex(ins[:n_chk], pool0[slot], L, budget, gpu_pair)
+        per_pair = 2 * dk * dv * 4 + L * (es * (2 * dk + 2 * dv) + gate_bytes_per_token_head(form, dk, es) + 4)
+        return dict(step=step, units=N * L, bytes=N * H * per_pair + (4 * N if indexed else 0),
+                    flops=N * L * H * 7 * dk * dv, kernel_key="decode", launches=1, parity=parity,
+                    hold=(dev_in, pool, out))
+    inp = make_form_inputs(w["B"], w["T"], w["H"], w["dk"], w["dv"], w["dtype"], rank_seed(w["index"], rank),
+                           form, state=w["state"], varlen=w["varlen"], raw=raw, gates=w["gates"],
+                           spread="default")
+    d = to_torch(inp, device)
+    if name == "prefill_bwd":
+        return setup_backward(inp, d, device)
+    out = torch.empty(d["v"].shape, dtype=d["q"].dtype, device=device)
+    Sf = torch.empty((inp.n_seqs, inp.H, inp.dk, inp.dv), dtype=torch.float32, device=device)
+    gate = d["f"] if form == "fused" else d["log_alpha"]
+
+    def step(i):
+        kda_chunk_fwd_ex(d["q"], d["k"], d["v"], gate, d["beta"], d["S0"], d["cu_seqlens"], out, Sf,
+                         gate_kind=kind, A_log=d["A_log"], dt_bias=d["dt_bias"], **flags)
+
+    def parity(budget):
+        return cpu_baseline(oracle_view(inp), budget, prefill_pairs(out, Sf, inp))
+    tok_heads = inp.total_tokens * inp.H
+    per_tok = es * (2 * inp.dk + 2 * inp.dv) + gate_bytes_per_token_head(form, inp.dk, es) + 4
+    states = inp.n_seqs * inp.H * inp.dk * inp.dv * 4 * ((inp.S0 is not None) + 1)
+    params = 2 * inp.H * inp.dk * 4 if form == "fused" else 0
+    return dict(step=step, units=inp.total_tokens, bytes=tok_heads * per_tok + states + params,
+                flops=alg_flops_prefill(tok_heads, inp.dk, inp.dv), kernel_key="chunk",
+                launches=2 + (inp.cu_seqlens is not None), parity=parity, hold=(d, out, Sf))
+
+
+def setup_backward(inp, d, device):
+    """The backward pass (kda_chunk_bwd) on a prefill workload: dO and dS_final drawn from
+    N(0, 1); parity of every gradient on a bounded oracle sample."""
+    import torch
+    from gated_delta_rule_119_b200 import kda_chunk_bwd
+    rng = np.random.default_rng([int(inp.meta["seed"]) if np.ndim(inp.meta["seed"]) == 0 else 0, 99])
+    dO = rng.standard_normal((inp.total_tokens, inp.H, inp.dv), dtype=np.float32)
+    dO_t = torch.from_numpy(dO).to(device).to(d["q"].dtype).view(d["v"].shape)
+    dO_bits = dO_t.view(-1).view(torch.int16).cpu().numpy().view(np.uint16).reshape(dO.shape) \
+        if inp.dtype == "bf16" else dO
+    dSf = rng.standard_normal((inp.n_seqs, inp.H, inp.dk, inp.dv), dtype=np.float32)
+    dSf_t = torch.from_numpy(dSf).to(device)
+    holder = {}
+
+    def step(i):
+        holder["g"] = kda_chunk_bwd(d["q"], d["k"], d["v"], d["log_alpha"], d["beta"], dO_t, d["S0"],
+                                    d["cu_seqlens"], dSf_t)
+
+    def parity(budget):
+        return cpu_baseline_backward(inp, dO_bits, dSf, holder, budget)
+    tok_heads = inp.total_tokens * inp.H
+    es = 2 if inp.dtype == "bf16" else 4
+    # read q, k, v, log_alpha, beta, dO (+ dS_final, S0); write dq, dk, dv, dlog_alpha, dbeta, dS0
+    per_tok = es * (3 * inp.dk + 2 * inp.dv) + es * (2 * inp.dk + inp.dv) + 2 * 4 * inp.dk + 2 * 4
+    states = inp.n_seqs * inp.H * inp.dk * inp.dv * 4 * (2 + (inp.S0 is not None))
+    return dict(step=step, units=inp.total_tokens, bytes=tok_heads * per_tok + states,
+                flops=alg_flops_backward(tok_heads, inp.dk, inp.dv), kernel_key="chunk_bwd",
+                launches=2, parity=parity, hold=(d, dO_t, dSf_t, holder), bound="alu")
 
 
 def time_steps(step, steps, warmup, device, stream, min_timed_s=1.0, min_passes=5,
@@ -410,6 +652,14 @@ def launch_duration_ms(step, n, device, stream):
 
 
 def roofline_entry(wl, launch_ms, hbm, peak_kind, name):
+    if wl.get("bound") == "alu":
+        achieved = wl["flops"] / (launch_ms / 1e3) / 1e12
+        return {"bound": "alu", "achieved": achieved, "peak": FP32_PEAK_TFLOPS, "unit": "TFLOP/s",
+                "frac": achieved / FP32_PEAK_TFLOPS, "traffic": None,
+                "peak_kind": "fp32 FMA peak from the unit counts (148 SMs x 128 lanes x 2 x 1.965 GHz)",
+                "kernel": "kda_chunk_bwd_kernel + kda_chunk_bwd_reduce_kernel (one kda_chunk_bwd call)",
+                "alg_flops_per_launch": wl["flops"], "alg_bytes_per_launch": wl["bytes"],
+                "hbm_frac": wl["bytes"] / (launch_ms / 1e3) / 1e9 / hbm, "launch_ms": launch_ms}
     achieved = wl["bytes"] / (launch_ms / 1e3) / 1e9
     return {"bound": "hbm", "achieved": achieved, "peak": hbm, "unit": "GB/s",
             "frac": achieved / hbm, "traffic": profiled_traffic(wl["kernel_key"], name),
@@ -417,7 +667,7 @@ def roofline_entry(wl, launch_ms, hbm, peak_kind, name):
             "kernel": {"chunk": "kda_chunk_intra_kernel + kda_chunk_scan_kernel "
                                 "(one kda_chunk_fwd call)",
                        "chunk_simt": "kda_chunk_simt_kernel",
-                       "decode": "kda_decode_kernel"}[wl["kernel_key"]],
+                       "decode": "kda_decode_step_kernel (one token) / kda_decode_kernel (general)"}[wl["kernel_key"]],
             "alg_bytes_per_launch": wl["bytes"], "launch_ms": launch_ms}
 
 
@@ -480,6 +730,13 @@ def run_ours(args, rank, local_rank, world):
     return res
 
 
+def variant_config(name):
+    base, form, raw, L, indexed = VARIANTS[name]
+    return {**workload_config(base, None, 1), "variant": name, "gate_form": form,
+            "in_kernel_norm_and_beta_logits": raw, "decode_tokens_per_call": L,
+            "indexed_state_pool": indexed}
+
+
 def run_other_workload(name, args, device, stream, rank, hbm, peak_kind):
     """One more workload in the same process: ms per step (median of timed passes), tokens/s,
     its roofline and parity on a bounded oracle sample.  Failures are reported, not raised."""
@@ -490,14 +747,13 @@ def run_other_workload(name, args, device, stream, rank, hbm, peak_kind):
         passes = time_steps(wl["step"], steps, 3, device, stream, min_timed_s=0.3, sampler=clk)
         launch_ms = launch_duration_ms(wl["step"], min(steps, 10), device, stream)
         ms = statistics.median(passes)
-        w = WORKLOADS[name]
         entry = {"ms_per_step": ms, "min_ms": min(passes), "max_ms": max(passes),
                  "passes": len(passes), "steps_per_pass": steps,
                  "value": wl["units"] / (ms / 1e3), "unit": "tokens/s",
                  "tflops": wl["flops"] / (launch_ms / 1e3) / 1e12,
                  "roofline": roofline_entry(wl, launch_ms, hbm, peak_kind, name),
                  "clocks": clk.summary(), "gpu_launches_per_step": wl["launches"],
-                 "config": workload_config(name, None, 1)}
+                 "config": variant_config(name) if name in VARIANTS else workload_config(name, None, 1)}
         if not args.no_cpu_baseline:
             cb = wl["parity"](args.workload_parity_budget)
             entry["parity"] = cb.pop("parity", None)
@@ -505,7 +761,7 @@ def run_other_workload(name, args, device, stream, rank, hbm, peak_kind):
         del wl
         return entry
     except Exception as e:  # noqa: BLE001 - reported in the line instead
-        return {"error": repr(e)[:300], "dtype": WORKLOADS[name]["dtype"]}
+        return {"error": repr(e)[:300]}
 
 
 def prefill_pairs(out, S_final, inp):
@@ -641,7 +897,9 @@ def main(argv=None):
     ap.add_argument("--min-timed-s", type=float, default=1.0,
                     help="repeat the timed passes of --steps steps until about this much "
                          "timed work (at least 5 passes)")
-    ap.add_argument("--workloads", default="decode,varlen,extremes",
+    ap.add_argument("--workloads",
+                    default="decode,varlen,extremes,prefill_fused,prefill_gdn,prefill_bwd,decode_indexed,"
+                            "decode_mtp4",
                     help="other workloads measured in the same process at N=1 (comma list; "
                          "empty for none)")
     ap.add_argument("--workload-parity-budget", type=float, default=3.0)

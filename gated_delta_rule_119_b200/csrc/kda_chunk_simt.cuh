@@ -89,7 +89,8 @@ __global__ void __launch_bounds__(kSimtThreads, 1) kda_chunk_simt_kernel(KdaChun
                 const size_t off = ((size_t)(c0 + r) * H + h) * DK + c;
                 kv = kda::to_f32(kg[off]);
                 qv = kda::to_f32(qg[off]);
-                lv = a.log_alpha[off];
+                lv = kda::gate_log_alpha<Tin>(a.gate_kind, a.gate, a.A_log, a.dt_bias,
+                                              (size_t)(c0 + r) * H + h, h, c, DK);
             }
             Kb[r * LKV + c] = kv;
             Qb[r * LK + c] = qv;
@@ -100,10 +101,32 @@ __global__ void __launch_bounds__(kSimtThreads, 1) kda_chunk_simt_kernel(KdaChun
             Vb[r * LV + c] = r < nr ? kda::to_f32(vg[((size_t)(c0 + r) * H + h) * DV + c]) : 0.f;
         }
         for (int r = tid; r < CH; r += kSimtThreads)
-            bt[r] = r < nr ? a.beta[(size_t)(c0 + r) * H + h] : 0.f;
+            bt[r] = r < nr ? kda::beta_of(a.beta[(size_t)(c0 + r) * H + h], a.flags) : 0.f;
         __syncthreads();
 
-        // 2. alpha = exp(log_alpha), in place.
+        // 2. unit-length keys / queries (KDA_NORM_K / KDA_NORM_Q), one warp per row, in place.
+        if (a.flags & (kda::FLAG_NORM_K | kda::FLAG_NORM_Q)) {
+            const int warp = tid >> 5, lane = tid & 31;
+            for (int r = warp; r < CH; r += kSimtThreads / 32) {
+                float kk = 0.f, qq = 0.f;
+                for (int c = lane; c < DK; c += 32) {
+                    kk = fmaf(Kb[r * LKV + c], Kb[r * LKV + c], kk);
+                    qq = fmaf(Qb[r * LK + c], Qb[r * LK + c], qq);
+                }
+#pragma unroll
+                for (int o = 16; o > 0; o >>= 1) {
+                    kk += __shfl_xor_sync(0xffffffffu, kk, o);
+                    qq += __shfl_xor_sync(0xffffffffu, qq, o);
+                }
+                const float fk = (a.flags & kda::FLAG_NORM_K) ? 1.f / fmaxf(sqrtf(kk), 1e-12f) : 1.f;
+                const float fq = (a.flags & kda::FLAG_NORM_Q) ? 1.f / fmaxf(sqrtf(qq), 1e-12f) : 1.f;
+                for (int c = lane; c < DK; c += 32) {
+                    Kb[r * LKV + c] *= fk;
+                    Qb[r * LK + c] *= fq;
+                }
+            }
+        }
+        //    alpha = exp(log_alpha), in place.
         for (int idx = tid; idx < CH * DK; idx += kSimtThreads) {
             const int r = idx / DK, c = idx % DK;
             Gb[r * LK + c] = expf(Gb[r * LK + c]);

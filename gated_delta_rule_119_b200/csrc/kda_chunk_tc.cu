@@ -84,7 +84,10 @@ constexpr uint32_t I_GC = I_BETA + 256; // [128]
 constexpr uint32_t I_BS = I_GC + 512;   // [4][128] sum of log_alpha per 16-row block
 constexpr uint32_t I_BT = I_BS + 2048;  // [4][128] product of alpha per block
 constexpr uint32_t I_XT = I_BT + 2048;  // [6][128] forward-substitution scratch
-constexpr uint32_t I_END = I_XT + 3072;
+constexpr uint32_t I_RK = I_XT + 3072;  // [64] 1 / ||k_r|| (unit-length keys), else unused
+constexpr uint32_t I_RQ = I_RK + 256;   // [64] 1 / ||q_r|| (unit-length queries), else unused
+constexpr uint32_t I_LA = I_RQ + 256;   // [64] the scalar gate's log alpha per row
+constexpr uint32_t I_END = I_LA + 256;
 constexpr size_t kIntraSmem = I_END + 1024;
 static_assert(I_TP % 1024 == 0 && I_KC % 1024 == 0, "tile alignment");
 static_assert(I_CA + 4096 <= I_TP, "block-path scratch inside T");
@@ -114,6 +117,14 @@ __device__ __forceinline__ uint4 pack8(const float *v) {
     return pk;
 }
 
+// x scaled by the row's unit-length factor (NORM) or unchanged.
+template <bool NORM>
+__device__ __forceinline__ float2 row_scaled(float2 x, const float *f, int r) {
+    if (!NORM) return x;
+    const float s = f[r];
+    return make_float2(x.x * s, x.y * s);
+}
+
 // Byte offset of element (r, c) of a [64][128] bf16 tile stored as two 64-column halves of
 // 128-byte rows, the 16-byte chunks of row r XOR-swizzled by r & 7 (the layout a TMA load with
 // 128-byte swizzle writes): conflict-free both for a warp reading 32 consecutive channels of one
@@ -126,20 +137,26 @@ __device__ __forceinline__ uint32_t rm_sw(int r, int c) {
 // offsets), and order[0..N) = the sequences by decreasing length (ties by index), so the scan
 // starts its longest chains first.  Up to kSortMax sequences are ranked; beyond that the order
 // is the identity.
+// Well-formed offsets need at most ceil(T_total / 64) + N slots, the workspace's size.  Offsets
+// that are not non-decreasing can make clamped sequences overlap and ask for more; the running
+// sum is therefore capped at max_slots, so a sequence gets min(its chunks, the slots left), and
+// the scan walks only base[n + 1] - base[n] chunks of sequence n: no slot outside the workspace
+// is ever written or read (the results of such a call are unspecified).
 constexpr int kSortMax = 256;
 
 __global__ void __launch_bounds__(kSortMax) kda_chunk_slots_kernel(const int32_t *cu_seqlens, int N,
-                                                                    int64_t T_total, int32_t *base,
-                                                                    int32_t *order) {
+                                                                    int64_t T_total, int64_t max_slots,
+                                                                    int32_t *base, int32_t *order) {
     if (threadIdx.x == 0) {
-        int32_t acc = 0;
+        int64_t acc = 0;
         for (int n = 0; n < N; ++n) {
             int64_t t0, t1;
             kda::seq_bounds(cu_seqlens, n, 0, T_total, t0, t1);
-            base[n] = acc;
-            acc += (int32_t)((t1 - t0 + CH - 1) / CH);
+            base[n] = (int32_t)acc;
+            const int64_t want = (t1 - t0 + CH - 1) / CH;
+            acc += want < max_slots - acc ? want : max_slots - acc;
         }
-        base[N] = acc;
+        base[N] = (int32_t)acc;
     }
     if (N > kSortMax) {
         for (int n = threadIdx.x; n < N; n += blockDim.x) order[n] = n;
@@ -160,33 +177,76 @@ __global__ void __launch_bounds__(kSortMax) kda_chunk_slots_kernel(const int32_t
     }
 }
 
-// Exact diagonal-block contribution of one channel whose decay over a 16-row block is too
-// strong for the rescaled factors: running products of alpha, inputs re-read from memory.
-// Adds beta_r k_r k_i D_ri to A (i < r) and s q_r k_i D_ri to the block's exact P sums.
-__device__ __noinline__ void exact_diag_channel(const KdaChunkArgs &a, int64_t c0, int nr, int h, int blk,
-                                                int ch, const float *sBeta, float *sCA, float *sCP) {
+// Exact diagonal-block contributions of the channels whose decay over a 16-row block is too
+// strong for the rescaled factors (-sum log_alpha over the block > kSpreadLimit): running
+// products of alpha, inputs re-read from memory.  Thread t takes block t / 64, column
+// i = (t / 4) % 16, the row half rh = (t / 2) % 2 (rows 8 rh .. 8 rh + 7 of the block) and the
+// channel half t % 2: over its flagged channels, in channel order, it carries the running
+// product D_Ri from row i down its rows; then the two channel halves of (block, i, rh) --
+// adjacent lanes -- are added.  Writes sCA[blk][R][i] = sum beta_R k_R k_i D_Ri (i < R) and
+// sCP[blk][R][i] = sum s q_R k_i D_Ri (i <= R) for the rows of the chunk, the same on every run.
+// Called by all NTHR threads of the CTA.  With NORM, k and q are scaled by the rows' unit-length
+// factors sRk, sRq.
+template <int GATE, bool NORM>
+__device__ __noinline__ void exact_diag_blocks(const KdaChunkArgs &a, int64_t c0, int nr, int h, const float *sBS,
+                                               const float *sBeta, const float *sRk, const float *sRq,
+                                               float *sCA, float *sCP) {
     const int H = a.H;
     const __nv_bfloat16 *qg = static_cast<const __nv_bfloat16 *>(a.q);
     const __nv_bfloat16 *kg = static_cast<const __nv_bfloat16 *>(a.k);
-    for (int i = 0; i < 16; ++i) {
-        const int I = 16 * blk + i;
-        if (I >= nr) break;
-        const float ki = __bfloat162float(kg[((size_t)(c0 + I) * H + h) * DK + ch]);
-        float f = 1.f;
-        for (int R = I; R < 16 * blk + 16 && R < nr; ++R) {
-            const size_t off = ((size_t)(c0 + R) * H + h) * DK + ch;
-            if (R > I) f *= __expf(a.log_alpha[off]);
-            const float kd = ki * f;
-            if (R > I) atomicAdd(&sCA[blk * 256 + (R - 16 * blk) * 16 + i], sBeta[R] * __bfloat162float(kg[off]) * kd);
-            atomicAdd(&sCP[blk * 256 + (R - 16 * blk) * 16 + i], a.scale * __bfloat162float(qg[off]) * kd);
+    const int t = threadIdx.x, chh = t & 1, rh = (t >> 1) & 1, i = (t >> 2) & 15, blk = t >> 6;
+    const int I = 16 * blk + i;
+    float sa[8], sp[8];
+#pragma unroll
+    for (int r = 0; r < 8; ++r) sa[r] = sp[r] = 0.f;
+    if (I < nr && 8 * rh + 7 >= i) {
+        for (int cc = 0; cc < DK / 2; ++cc) {
+            const int ch = (DK / 2) * chh + cc;
+            if (!(sBS[blk * 128 + ch] < -kSpreadLimit)) continue;
+            float ki = __bfloat162float(kg[((size_t)(c0 + I) * H + h) * DK + ch]);
+            if (NORM) ki *= sRk[I];
+            float f = 1.f;
+            for (int R = i + 1; R < 8 * rh && 16 * blk + R < nr; ++R)   // rows before this half
+                f *= __expf(kda::gate_log_alpha<__nv_bfloat16>(GATE, a.gate, a.A_log, a.dt_bias,
+                                                                (size_t)(c0 + 16 * blk + R) * H + h, h, ch, DK));
+#pragma unroll
+            for (int r = 0; r < 8; ++r) {
+                const int R = 8 * rh + r, Rg = 16 * blk + R;
+                if (R >= i && Rg < nr) {
+                    const size_t th = (size_t)(c0 + Rg) * H + h, off = th * DK + ch;
+                    if (R > i)
+                        f *= __expf(kda::gate_log_alpha<__nv_bfloat16>(GATE, a.gate, a.A_log, a.dt_bias, th, h, ch, DK));
+                    const float kd = ki * f;
+                    const float kr = __bfloat162float(kg[off]) * (NORM ? sRk[Rg] : 1.f);
+                    const float qr = __bfloat162float(qg[off]) * (NORM ? sRq[Rg] : 1.f);
+                    if (R > i) sa[r] += sBeta[Rg] * kr * kd;
+                    sp[r] += a.scale * qr * kd;
+                }
+            }
+        }
+    }
+#pragma unroll
+    for (int r = 0; r < 8; ++r) {
+        sa[r] += __shfl_xor_sync(0xffffffffu, sa[r], 1);
+        sp[r] += __shfl_xor_sync(0xffffffffu, sp[r], 1);
+    }
+    if (chh == 0) {
+#pragma unroll
+        for (int r = 0; r < 8; ++r) {
+            sCA[blk * 256 + (8 * rh + r) * 16 + i] = sa[r];
+            sCP[blk * 256 + (8 * rh + r) * 16 + i] = sp[r];
         }
     }
 }
 
 // ======================================================================= intra-chunk kernel
+// GATE: the gate form (kda_gate_kind); NORM: unit-length keys and/or queries (per a.flags).
+// tmap_g is the gate tile map: log_alpha [64][128] fp32 (CHANNEL) or f [64][128] bf16
+// (FUSED); the scalar gate is read like beta, and no gate is read without decay.
+template <int GATE, bool NORM>
 __global__ void __launch_bounds__(NTHR, 2)
     kda_chunk_intra_kernel(KdaChunkArgs a, uint8_t *ws, const int32_t *slot_base,
-                           const __grid_constant__ CUtensorMap tmap_la, const __grid_constant__ CUtensorMap tmap_k,
+                           const __grid_constant__ CUtensorMap tmap_g, const __grid_constant__ CUtensorMap tmap_k,
                            const __grid_constant__ CUtensorMap tmap_q) {
     extern __shared__ uint8_t smraw[];
     uint8_t *sm = smraw + ((1024u - (smem_u32(smraw) & 1023u)) & 1023u);   // stays a shared-space pointer
@@ -227,13 +287,15 @@ __global__ void __launch_bounds__(NTHR, 2)
     float *sSC = (float *)(sm + I_SC), *sCP = (float *)(sm + I_CP), *sCA = (float *)(sm + I_CA);
     float *sBeta = (float *)(sm + I_BETA), *sGC = (float *)(sm + I_GC);
     float *sBS = (float *)(sm + I_BS), *sBT = (float *)(sm + I_BT), *sXT = (float *)(sm + I_XT);
+    float *sRk = (float *)(sm + I_RK), *sRq = (float *)(sm + I_RQ), *sLa = (float *)(sm + I_LA);
     const float scale = a.scale;
 
-    // The chunk's inputs by TMA, issued by one thread: log_alpha [64][128] fp32 into the space of
-    // [k gamma; s q gamma] and k [64][128] bf16 into the space of the update operand (both
-    // row-major; pass 1 moves them to registers before pass 2 overwrites them), q as two
-    // 64-column halves in the rm_sw layout into the space of [T'; P T'].  Rows past the chunk's
-    // end hold the next tokens (zeros past the last token) and are masked where they are read.
+    // The chunk's inputs by TMA, issued by one thread: the gate tile (log_alpha [64][128] fp32,
+    // or f [64][128] bf16) into the space of [k gamma; s q gamma] and k [64][128] bf16 into the
+    // space of the update operand (both row-major; pass 1 moves them to registers before pass 2
+    // overwrites them), q as two 64-column halves in the rm_sw layout into the space of
+    // [T'; P T'].  Rows past the chunk's end hold the next tokens (zeros past the last token)
+    // and are masked where they are read.
     uint8_t *sQ = sTP;
     if (tid == 0) {
         mbar_init(&bar_ap, 1);
@@ -242,26 +304,73 @@ __global__ void __launch_bounds__(NTHR, 2)
         mbar_init(&bar_in, 1);
         mbar_init_fence();
         s_abort = 0;
-        mbar_arrive_expect_tx(&bar_in, 65536);
-        tma_load_3d(sKQ, &tmap_la, 0, h, (int)c0, &bar_in);
+        constexpr uint32_t gate_bytes = GATE == kda::GATE_CHANNEL ? 32768u : (GATE == kda::GATE_FUSED ? 16384u : 0u);
+        mbar_arrive_expect_tx(&bar_in, 32768u + gate_bytes);
+        if (gate_bytes) tma_load_3d(sKQ, &tmap_g, 0, h, (int)c0, &bar_in);
         tma_load_3d(sKC, &tmap_k, 0, h, (int)c0, &bar_in);
         tma_load_3d(sQ, &tmap_q, 0, h, (int)c0, &bar_in);
         tma_load_3d(sQ + 8192, &tmap_q, 64, h, (int)c0, &bar_in);
     }
-    if (tid < CH) sBeta[tid] = tid < nr ? a.beta[(size_t)(c0 + tid) * H + h] : 0.f;
+    if (tid < CH) {
+        sBeta[tid] = tid < nr ? kda::beta_of(a.beta[(size_t)(c0 + tid) * H + h], a.flags) : 0.f;
+        if (GATE == kda::GATE_SCALAR)
+            sLa[tid] = tid < nr ? static_cast<const float *>(a.gate)[(size_t)(c0 + tid) * H + h] : 0.f;
+    }
     if (warp == 0) tmem_alloc(&s_tmem, 256);
     __syncthreads();                     // the barriers are initialised before anyone waits
     if (!mbar_wait(&bar_in, 0, kWaitCycles)) s_abort = 1;
+
+    // Unit-length keys / queries: 1 / ||x_r|| per row, four threads per row (k row-major in the
+    // update operand's space, q in the rm_sw layout); read in pass 2 after pass 1's barrier.
+    if (NORM) {
+        const int r = tid >> 2, qd = tid & 3;
+        float kk = 0.f, qq = 0.f;
+#pragma unroll
+        for (int m = 0; m < 4; ++m) {
+            const uint4 kw = *(const uint4 *)(sKC + r * 256 + qd * 64 + m * 16);
+            const uint4 qw = *(const uint4 *)(sQ + (qd >> 1) * 8192 + r * 128 + ((((qd & 1) * 4 + m) ^ (r & 7)) << 4));
+            const uint32_t kk4[4] = {kw.x, kw.y, kw.z, kw.w}, qq4[4] = {qw.x, qw.y, qw.z, qw.w};
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                const float2 x = unpack_bf16(kk4[e]), y = unpack_bf16(qq4[e]);
+                kk = fmaf(x.x, x.x, fmaf(x.y, x.y, kk));
+                qq = fmaf(y.x, y.x, fmaf(y.y, y.y, qq));
+            }
+        }
+        kk += __shfl_xor_sync(0xffffffffu, kk, 1);
+        kk += __shfl_xor_sync(0xffffffffu, kk, 2);
+        qq += __shfl_xor_sync(0xffffffffu, qq, 1);
+        qq += __shfl_xor_sync(0xffffffffu, qq, 2);
+        if (qd == 0) {
+            sRk[r] = (a.flags & kda::FLAG_NORM_K) ? 1.f / fmaxf(sqrtf(kk), 1e-12f) : 1.f;
+            sRq[r] = (a.flags & kda::FLAG_NORM_Q) ? 1.f / fmaxf(sqrtf(qq), 1e-12f) : 1.f;
+        }
+    }
 
     // E2 thread mapping: channels {c2, c2 + 1} of 16-row block eb.
     const int c2 = 2 * (tid & 63), eb = tid >> 6;
     float2 la[16];
     uint32_t kr2[16];
+    float2 alog = make_float2(0.f, 0.f), dtb = make_float2(0.f, 0.f);
+    if (GATE == kda::GATE_FUSED) {
+        alog = *reinterpret_cast<const float2 *>(a.A_log + (size_t)h * DK + c2);
+        dtb = *reinterpret_cast<const float2 *>(a.dt_bias + (size_t)h * DK + c2);
+    }
 #pragma unroll
     for (int rr = 0; rr < 16; ++rr) {
         const int r = 16 * eb + rr;
         const bool ok = r < nr;
-        la[rr] = ok ? *reinterpret_cast<const float2 *>(sKQ + 4 * (r * DK + c2)) : make_float2(0.f, 0.f);
+        if (GATE == kda::GATE_CHANNEL) {
+            la[rr] = ok ? *reinterpret_cast<const float2 *>(sKQ + 4 * (r * DK + c2)) : make_float2(0.f, 0.f);
+        } else if (GATE == kda::GATE_FUSED) {
+            const float2 f = unpack_bf16(*reinterpret_cast<const uint32_t *>(sKQ + 2 * (r * DK + c2)));
+            la[rr] = ok ? make_float2(kda::fused_log_alpha(f.x, alog.x, dtb.x), kda::fused_log_alpha(f.y, alog.y, dtb.y))
+                        : make_float2(0.f, 0.f);
+        } else if (GATE == kda::GATE_SCALAR) {
+            la[rr] = make_float2(sLa[r], sLa[r]);
+        } else {
+            la[rr] = make_float2(0.f, 0.f);
+        }
         kr2[rr] = ok ? *reinterpret_cast<const uint32_t *>(sKC + 2 * (r * DK + c2)) : 0u;
     }
 
@@ -331,8 +440,8 @@ __global__ void __launch_bounds__(NTHR, 2)
                 const int r = 16 * eb + rr;
                 l0 *= la[rr].x;
                 l1 *= la[rr].y;
-                const float2 kv = unpack_bf16(kr2[rr]);
-                const float2 qv = unpack_bf16(r < nr ? *(const uint32_t *)(sQ + rm_sw(r, c2)) : 0u);
+                const float2 kv = row_scaled<NORM>(unpack_bf16(kr2[rr]), sRk, r);
+                const float2 qv = row_scaled<NORM>(unpack_bf16(r < nr ? *(const uint32_t *)(sQ + rm_sw(r, c2)) : 0u), sRq, r);
                 const float g0 = gpre.x * l0, g1 = gpre.y * l1;
                 *(uint32_t *)(sKQ + col_kq + sw128(r, c2 & 63)) = pack_bf16(kv.x * g0, kv.y * g1);
                 *(uint32_t *)(sKQ + col_kq + sw128(64 + r, c2 & 63)) = pack_bf16(scale * qv.x * g0, scale * qv.y * g1);
@@ -341,42 +450,49 @@ __global__ void __launch_bounds__(NTHR, 2)
 #pragma unroll
             for (int rr = 15; rr >= 0; --rr) {
                 const int r = 16 * eb + rr;
-                const float2 kv = unpack_bf16(kr2[rr]);
+                const float2 kv = row_scaled<NORM>(unpack_bf16(kr2[rr]), sRk, r);
                 *(uint32_t *)(sKC + col_kc + sw128(r, c2 & 63)) =
                     pack_bf16(kv.x * (g0 * ksuf.x), kv.y * (g1 * ksuf.y));
                 g0 *= la[rr].x;
                 g1 *= la[rr].y;
             }
         } else {
-            float l0 = 1.f, l1 = 1.f;
+            // The rescaled factors rho * (prefix product) and rho * (suffix product) are carried
+            // as running products that start at rho: they stay in [e^-70, e^70] for a block
+            // spread up to kSpreadLimit, where the unscaled products alone would leave fp32's
+            // normal range (below e^-87) for spreads past 87 before rho could scale them back.
+            float l0 = 1.f, l1 = 1.f, m0 = rho0, m1 = rho1;
 #pragma unroll
             for (int rr = 0; rr < 16; ++rr) {
                 const int r = 16 * eb + rr;
                 l0 *= la[rr].x;
                 l1 *= la[rr].y;
-                const float2 kv = unpack_bf16(kr2[rr]);
-                const float2 qv = unpack_bf16(r < nr ? *(const uint32_t *)(sQ + rm_sw(r, c2)) : 0u);
+                m0 *= la[rr].x;
+                m1 *= la[rr].y;
+                const float2 kv = row_scaled<NORM>(unpack_bf16(kr2[rr]), sRk, r);
+                const float2 qv = row_scaled<NORM>(unpack_bf16(r < nr ? *(const uint32_t *)(sQ + rm_sw(r, c2)) : 0u), sRq, r);
                 const float g0 = gpre.x * l0, g1 = gpre.y * l1;
                 *(uint32_t *)(sKQ + col_kq + sw128(r, c2 & 63)) = pack_bf16(kv.x * g0, kv.y * g1);
                 *(uint32_t *)(sKQ + col_kq + sw128(64 + r, c2 & 63)) = pack_bf16(scale * qv.x * g0, scale * qv.y * g1);
-                *(uint32_t *)(sKL + rm_sw(r, c2)) = pack_bf16(kv.x * (rho0 * l0), kv.y * (rho1 * l1));
-                *(uint32_t *)(sQ + rm_sw(r, c2)) =
-                    pack_bf16(scale * qv.x * (rho0 * l0), scale * qv.y * (rho1 * l1));
+                *(uint32_t *)(sKL + rm_sw(r, c2)) = pack_bf16(kv.x * m0, kv.y * m1);
+                *(uint32_t *)(sQ + rm_sw(r, c2)) = pack_bf16(scale * qv.x * m0, scale * qv.y * m1);
             }
-            float g0 = 1.f, g1 = 1.f;
+            float g0 = 1.f, g1 = 1.f, n0 = rho0, n1 = rho1;
 #pragma unroll
             for (int rr = 15; rr >= 0; --rr) {
                 const int r = 16 * eb + rr;
-                const float2 kv = unpack_bf16(kr2[rr]);
+                const float2 kv = row_scaled<NORM>(unpack_bf16(kr2[rr]), sRk, r);
                 *(uint32_t *)(gslot + SLOT_KC + col_kc + sw128(r, c2 & 63)) =
                     pack_bf16(kv.x * (g0 * ksuf.x), kv.y * (g1 * ksuf.y));
-                *(uint32_t *)(sKR + rm_sw(r, c2)) = pack_bf16(kv.x * (rho0 * g0), kv.y * (rho1 * g1));
+                *(uint32_t *)(sKR + rm_sw(r, c2)) = pack_bf16(kv.x * n0, kv.y * n1);
                 g0 *= la[rr].x;
                 g1 *= la[rr].y;
+                n0 *= la[rr].x;
+                n1 *= la[rr].y;
             }
         }
-        if (!fast && fl0) exact_diag_channel(a, c0, nr, h, eb, c2, sBeta, sCA, sCP);
-        if (!fast && fl1) exact_diag_channel(a, c0, nr, h, eb, c2 + 1, sBeta, sCA, sCP);
+        if (!fast && __syncthreads_or(fl0 || fl1))
+            exact_diag_blocks<GATE, NORM>(a, c0, nr, h, sBS, sBeta, sRk, sRq, sCA, sCP);
         if (eb == 0) {
             float2 gc = make_float2(1.f, 1.f);
 #pragma unroll
@@ -746,8 +862,9 @@ __global__ void __launch_bounds__(SCAN_THREADS, 1)
     __nv_bfloat16 *og = static_cast<__nv_bfloat16 *>(a.out);
     int64_t t0, t1;
     kda::seq_bounds(a.cu_seqlens, n, a.T, a.T_total, t0, t1);
-    const int nchunks = (int)((t1 - t0 + CH - 1) / CH);
+    int nchunks = (int)((t1 - t0 + CH - 1) / CH);
     const int base = slot_base ? slot_base[n] : n * ((a.T + CH - 1) / CH);
+    if (slot_base && slot_base[n + 1] - base < nchunks) nchunks = slot_base[n + 1] - base;   // malformed offsets
     uint8_t *sS = sm + S_S;
 
     if (tid == 0) {
@@ -1002,11 +1119,32 @@ constexpr int kMaxDevices = 64;
 std::atomic<bool> g_configured[kMaxDevices] = {};
 std::atomic<bool> g_pool_configured[kMaxDevices] = {};
 
+using IntraKernel = void (*)(KdaChunkArgs, uint8_t *, const int32_t *, const CUtensorMap, const CUtensorMap,
+                             const CUtensorMap);
+
+// The intra-chunk kernel for a gate form and normalisation choice.
+IntraKernel intra_kernel_for(int gate_kind, bool norm) {
+    switch (gate_kind) {
+    case kda::GATE_SCALAR:
+        return norm ? kda_chunk_intra_kernel<kda::GATE_SCALAR, true> : kda_chunk_intra_kernel<kda::GATE_SCALAR, false>;
+    case kda::GATE_NONE:
+        return norm ? kda_chunk_intra_kernel<kda::GATE_NONE, true> : kda_chunk_intra_kernel<kda::GATE_NONE, false>;
+    case kda::GATE_FUSED:
+        return norm ? kda_chunk_intra_kernel<kda::GATE_FUSED, true> : kda_chunk_intra_kernel<kda::GATE_FUSED, false>;
+    default:
+        return norm ? kda_chunk_intra_kernel<kda::GATE_CHANNEL, true> : kda_chunk_intra_kernel<kda::GATE_CHANNEL, false>;
+    }
+}
+
 cudaError_t configure(int dev) {
     if (dev >= 0 && dev < kMaxDevices && g_configured[dev].load(std::memory_order_acquire)) return cudaSuccess;
-    cudaError_t e = cudaFuncSetAttribute(kda_chunk_intra_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         (int)kIntraSmem);
-    if (e != cudaSuccess) return e;
+    cudaError_t e = cudaSuccess;
+    for (int g = 0; g < 4; ++g)
+        for (int nm = 0; nm < 2; ++nm) {
+            e = cudaFuncSetAttribute(intra_kernel_for(g, nm != 0), cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                     (int)kIntraSmem);
+            if (e != cudaSuccess) return e;
+        }
     e = cudaFuncSetAttribute(kda_chunk_scan_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kScanSmem);
     if (e != cudaSuccess) return e;
     if (dev >= 0 && dev < kMaxDevices) g_configured[dev].store(true, std::memory_order_release);
@@ -1092,19 +1230,27 @@ cudaError_t kda_launch_chunk_tc_ws(const KdaChunkArgs &a, void *ws, cudaStream_t
     int32_t *slot_base = a.cu_seqlens ? static_cast<int32_t *>(ws) : nullptr;
     uint8_t *slots = static_cast<uint8_t *>(ws) + head_bytes_of(a);
     if (max_slots > 0) {
-        CUtensorMap tmap_la, tmap_k, tmap_q;
-        if ((e = encode_map(a, a.log_alpha, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, DK, CU_TENSOR_MAP_SWIZZLE_NONE,
-                            &tmap_la)) != cudaSuccess)
+        CUtensorMap tmap_g, tmap_k, tmap_q;
+        memset(&tmap_g, 0, sizeof(tmap_g));          // never read by the scalar and no-decay forms
+        if (a.gate_kind == kda::GATE_CHANNEL &&
+            (e = encode_map(a, a.gate, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, DK, CU_TENSOR_MAP_SWIZZLE_NONE,
+                            &tmap_g)) != cudaSuccess)
+            return e;
+        if (a.gate_kind == kda::GATE_FUSED &&
+            (e = encode_map(a, a.gate, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, DK, CU_TENSOR_MAP_SWIZZLE_NONE,
+                            &tmap_g)) != cudaSuccess)
             return e;
         if ((e = encode_map(a, a.k, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, DK, CU_TENSOR_MAP_SWIZZLE_NONE,
                             &tmap_k)) != cudaSuccess)
             return e;
         if ((e = encode_tok_map(a, a.q, &tmap_q)) != cudaSuccess) return e;
         if (a.cu_seqlens)
-            kda_chunk_slots_kernel<<<1, kSortMax, 0, stream>>>(a.cu_seqlens, a.N, a.T_total, slot_base,
-                                                                slot_base + a.N + 1);
+            kda_chunk_slots_kernel<<<1, kSortMax, 0, stream>>>(a.cu_seqlens, a.N, a.T_total, max_slots,
+                                                                slot_base, slot_base + a.N + 1);
         const dim3 grid((unsigned)max_slots, (unsigned)a.H);
-        kda_chunk_intra_kernel<<<grid, NTHR, kIntraSmem, stream>>>(a, slots, slot_base, tmap_la, tmap_k, tmap_q);
+        const bool norm = (a.flags & (kda::FLAG_NORM_K | kda::FLAG_NORM_Q)) != 0;
+        intra_kernel_for(a.gate_kind, norm)<<<grid, NTHR, kIntraSmem, stream>>>(a, slots, slot_base, tmap_g,
+                                                                                 tmap_k, tmap_q);
     }
     CUtensorMap tmap_v, tmap_o;
     if ((e = encode_tok_map(a, a.v, &tmap_v)) != cudaSuccess) return e;

@@ -35,27 +35,66 @@ __device__ __forceinline__ void seq_bounds(const int32_t *cu_seqlens, int n, int
     t1 = b;
 }
 
+// Gate forms and flags (the kda_gate_kind / kda_gate_flags values of include/kda.h).
+enum : int { GATE_CHANNEL = 0, GATE_SCALAR = 1, GATE_NONE = 2, GATE_FUSED = 3 };
+enum : int { FLAG_NORM_Q = 1, FLAG_NORM_K = 2, FLAG_BETA_LOGIT = 4 };
+constexpr float kFusedLogAlphaMin = -1e4f;   // alpha = e^-1e4 is 0 in fp32
+
+// ln(1 + e^x) in fp32: x itself once e^-x is below fp32 resolution.
+__device__ __forceinline__ float softplus(float x) { return x > 20.f ? x : log1pf(expf(x)); }
+
+// The fused gate of "Ten questions" Q9: log alpha = -exp(A_log) softplus(f + dt_bias).
+__device__ __forceinline__ float fused_log_alpha(float f, float A_log, float dt_bias) {
+    return fmaxf(-expf(A_log) * softplus(f + dt_bias), kFusedLogAlphaMin);
+}
+
+__device__ __forceinline__ float beta_of(float b, int flags) {
+    return (flags & FLAG_BETA_LOGIT) ? 1.f / (1.f + expf(-b)) : b;
+}
+
+// log alpha of channel c at token-head row th (= t * H + h) for any gate form; Tin is the
+// input dtype (the type of f for the fused form).
+template <typename Tin>
+__device__ __forceinline__ float gate_log_alpha(int kind, const void *gate, const float *A_log,
+                                                const float *dt_bias, size_t th, int h, int c, int dk) {
+    switch (kind) {
+    case GATE_CHANNEL: return static_cast<const float *>(gate)[th * dk + c];
+    case GATE_SCALAR: return static_cast<const float *>(gate)[th];
+    case GATE_FUSED:
+        return fused_log_alpha(to_f32(static_cast<const Tin *>(gate)[th * dk + c]), A_log[(size_t)h * dk + c],
+                               dt_bias[(size_t)h * dk + c]);
+    default: return 0.f;
+    }
+}
+
 }  // namespace kda
 
 // Host-side launchers (defined in the kernel files, called by kda_api.cu).
 struct KdaChunkArgs {
     const void *q, *k, *v;
-    const float *log_alpha, *beta, *S0;
+    const void *gate;                 // log_alpha (CHANNEL, SCALAR) or f (FUSED); NULL for NONE
+    const float *A_log, *dt_bias;     // [H, dk], FUSED only
+    const float *beta, *S0;
     const int32_t *cu_seqlens;
     void *out;
     float *S_final;
     int N, T, H, dk, dv;
     int64_t T_total;
     float scale;
+    int gate_kind, flags;
 };
 
 struct KdaDecodeArgs {
     const void *q, *k, *v;
-    const float *log_alpha, *beta;
-    float *S;
+    const void *gate;
+    const float *A_log, *dt_bias;
+    const float *beta;
+    float *S;                         // the state pool [P, H, dk, dv]
+    const int32_t *state_idx;         // [N] or NULL (slot n)
     void *out;
-    int N, H, dk, dv;
+    int N, L, H, dk, dv, P;
     float scale;
+    int gate_kind, flags;
 };
 
 cudaError_t kda_launch_decode(const KdaDecodeArgs &a, int dtype, cudaStream_t stream);
@@ -67,5 +106,10 @@ size_t kda_chunk_tc_workspace_bytes(const KdaChunkArgs &a);
 cudaError_t kda_launch_chunk_tc_ws(const KdaChunkArgs &a, void *ws, cudaStream_t stream);
 // Device address of the fixed scratch buffer of the current device (kda_noalloc.cu).
 cudaError_t kda_noalloc_scratch(void **ptr);
+size_t kda_chunk_bwd_workspace_bytes(const KdaChunkArgs &a);
+cudaError_t kda_launch_chunk_bwd(const KdaChunkArgs &a, int dtype, const void *dO, const float *dS_final,
+                                 void *dq, void *dk, void *dv, float *dgate, float *dbeta, float *dS0,
+                                 void *ws, cudaStream_t stream);
 cudaError_t kda_read_device_status(unsigned int *status, bool clear);
+cudaError_t kda_decode_read_status(unsigned int *status, bool clear);
 cudaError_t kda_launch_wait_selftest(int limit_us, cudaStream_t stream);

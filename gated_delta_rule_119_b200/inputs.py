@@ -19,6 +19,19 @@ Recipe (one numpy ``default_rng(seed)`` stream per workload, PCG64):
   heads [H/2, H) draw U(-6, -3) (strong forget), beta ~ U(0.95, 1);
 * S0 ~ N(0, 0.02) (standard deviation 0.02) when the workload carries a state.
 
+Gate forms of the extended entry points (``make_form_inputs``): the tensors above, then
+the form's own draws from a second stream of the same seed (``default_rng([*seed, 7])``):
+
+* "scalar" (Gated DeltaNet): log_alpha [T, H] = -softplus(N(0, 1)) per (token, head);
+* "none" (DeltaNet): no gate;
+* "fused": f [T, H, dk] ~ N(0, 1) in the storage dtype, A_log [H, dk] ~ U(-1, 1) and
+  dt_bias [H, dk] ~ N(0, 0.5) fp32 (log alpha = -exp(A_log) softplus(f + dt_bias) is formed
+  by the kernel; the per-channel decay spans a wide range, some channels forgetting several
+  times faster than the default gates); with ``spread="default"`` A_log = dt_bias = 0, so the
+  fused gate is -softplus(N(0, 1)), the default gates' distribution; with ``raw`` the keys
+  and queries stay unnormalised N(0, 1) draws (the kernel scales them) and beta is a
+  standard-normal logit (the kernel applies the sigmoid).
+
 Values are generated in fp32 (or fp64 and then rounded to fp32), then bf16
 inputs are rounded to nearest-even from that fp32 value.  The bf16 tensors are
 kept as their raw uint16 bit patterns so that every consumer sees the same
@@ -97,6 +110,11 @@ class KDAInputs:
     dv: int
     dtype: str
     meta: dict = field(default_factory=dict)
+    form: str = "channel"           # gate form: channel | scalar | none | fused
+    f: np.ndarray | None = None     # fused gate pre-activation [T_total, H, dk] (storage dtype)
+    A_log: np.ndarray | None = None     # [H, dk] fp32
+    dt_bias: np.ndarray | None = None   # [H, dk] fp32
+    flags: int = 0                  # NORM_Q | NORM_K | BETA_LOGIT of the extended entry points
 
     @property
     def n_seqs(self) -> int:
@@ -164,6 +182,43 @@ def make_inputs(B: int, T: int, H: int, dk: int, dv: int, dtype: str, seed,
                      H=H, dk=dk, dv=dv, dtype=dtype, meta=dict(seed=seed, gates=gates))
 
 
+def make_form_inputs(B: int, T: int, H: int, dk: int, dv: int, dtype: str, seed, form: str,
+                     state: bool = False, varlen: bool = False, cu_seqlens=None, raw: bool = False,
+                     gates: str = "default", spread: str = "wide") -> KDAInputs:
+    """One batch for a gate form of the extended entry points: the tensors of
+    :func:`make_inputs`, then the form's gate from a second stream of the seed (see the
+    module recipe).  ``raw`` (fused form only): unnormalised q, k and beta logits, with the flags
+    that ask the kernel to normalise and squash them."""
+    inp = make_inputs(B, T, H, dk, dv, dtype, seed, state=state, varlen=varlen, gates=gates,
+                      cu_seqlens=cu_seqlens)
+    rng = np.random.default_rng([*np.atleast_1d(np.asarray(seed, dtype=np.int64)).tolist(), 7])
+    Tt = inp.total_tokens
+    inp.form = form
+    if form == "channel":
+        return inp
+    if form == "scalar":
+        f = rng.standard_normal((Tt, H), dtype=np.float32).astype(np.float64)
+        inp.log_alpha = (-np.logaddexp(0.0, f)).astype(np.float32)
+    elif form == "none":
+        inp.log_alpha = None
+    elif form == "fused":
+        inp.log_alpha = None
+        inp.f = to_storage(rng.standard_normal((Tt, H, dk), dtype=np.float32), dtype)
+        inp.A_log = rng.uniform(-1.0, 1.0, size=(H, dk)).astype(np.float32)
+        inp.dt_bias = (0.5 * rng.standard_normal((H, dk))).astype(np.float32)
+        if spread == "default":
+            inp.A_log[:] = 0.0
+            inp.dt_bias[:] = 0.0
+        if raw:
+            inp.q = to_storage(rng.standard_normal((Tt, H, dk), dtype=np.float32), dtype)
+            inp.k = to_storage(rng.standard_normal((Tt, H, dk), dtype=np.float32), dtype)
+            inp.beta = rng.standard_normal((Tt, H), dtype=np.float32)
+            inp.flags = 1 | 2 | 4          # NORM_Q | NORM_K | BETA_LOGIT
+    else:
+        raise ValueError(f"unknown gate form {form!r}")
+    return inp
+
+
 def make_workload(name: str, **override) -> KDAInputs:
     """The named prefill workload at full size (``decode`` is built by
     :func:`make_decode_state` / :func:`make_decode_step`)."""
@@ -218,13 +273,17 @@ def to_torch(inp: KDAInputs, device="cuda", pin: bool = False) -> dict:
     d = {}
     for name in ("q", "k", "v"):
         d[name] = storage_to_torch(getattr(inp, name), inp.dtype, device, pin)
-    d["log_alpha"] = storage_to_torch(inp.log_alpha, "f32", device, pin)
+    d["log_alpha"] = None if inp.log_alpha is None else storage_to_torch(inp.log_alpha, "f32", device, pin)
     d["beta"] = storage_to_torch(inp.beta, "f32", device, pin)
+    d["f"] = None if inp.f is None else storage_to_torch(inp.f, inp.dtype, device, pin)
+    d["A_log"] = None if inp.A_log is None else storage_to_torch(inp.A_log, "f32", device, pin)
+    d["dt_bias"] = None if inp.dt_bias is None else storage_to_torch(inp.dt_bias, "f32", device, pin)
     d["S0"] = None if inp.S0 is None else storage_to_torch(inp.S0, "f32", device, pin)
     d["cu_seqlens"] = None if inp.cu_seqlens is None else \
         storage_to_torch(inp.cu_seqlens.astype(np.int32), "f32", device, pin)
     if inp.cu_seqlens is None and "step" not in inp.meta:
-        for name in ("q", "k", "v", "log_alpha", "beta"):
+        for name in ("q", "k", "v", "log_alpha", "beta", "f"):
             t = d[name]
-            d[name] = t.view(inp.B, inp.T, *t.shape[1:])
+            if t is not None:
+                d[name] = t.view(inp.B, inp.T, *t.shape[1:])
     return d

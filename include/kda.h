@@ -60,7 +60,9 @@ enum kda_status {
     KDA_ERR_ALIAS = -6,   /* an output overlaps an input it must not overlap */
     KDA_ERR_CUDA = -7,    /* a CUDA launch failed; kda_status_string names the CUDA error */
     KDA_ERR_TIMEOUT = -8, /* reserved for bounded device-side waits */
-    KDA_ERR_SCRATCH = -9  /* kda_chunk_fwd_noalloc: the workspace would exceed its fixed buffer */
+    KDA_ERR_SCRATCH = -9, /* kda_chunk_fwd_noalloc: the workspace would exceed its fixed buffer */
+    KDA_ERR_GATE = -10,   /* _ex entry points: a bad gate form, flag or gate pointer */
+    KDA_ERR_INDEX = -11   /* kda_device_status: a kda_decode_ex state index was >= the pool size */
 };
 
 /*
@@ -124,8 +126,10 @@ int kda_chunk_fwd(const void *q, const void *k, const void *v, const float *log_
  *    problem returns KDA_ERR_SCRATCH, found on the host before any CUDA call.  Only
  *    KDA_BF16 with dk = dv = 128 uses the buffer; every other case needs none.
  *  - The first call on a device looks up the buffer's device address (one CUDA runtime
- *    query, made with that device current) and keeps it.  A caller that records its
- *    calls into a stream capture should make one call on each device before it starts.
+ *    query, made with that device current) and keeps it for the life of the process.  A
+ *    caller that records its calls into a stream capture should make one call on each
+ *    device before it starts.  Resetting a device (cudaDeviceReset) after the first call
+ *    on it is not supported: the kept address may no longer be the buffer's.
  *  - Nothing in the buffer needs to start at zero: each call writes every byte of it
  *    that the call later reads.
  *  - Overlapping calls race: two calls on one device that can run at the same time
@@ -138,6 +142,84 @@ int kda_chunk_fwd_noalloc(const void *q, const void *k, const void *v, const flo
                           const float *beta, const float *S0, const int32_t *cu_seqlens,
                           void *out, float *S_final, int B, int T, int H, int dk, int dv, int C,
                           int dtype, kda_stream_t stream);
+
+/*
+ * Gate forms of the entry points with the _ex suffix.  Every form is the recurrence above
+ * with a different way of giving alpha_t (and, with flags, beta_t and unit-length q, k):
+ *
+ *  KDA_GATE_CHANNEL  gate = log_alpha [.., H, dk] fp32, one decay per channel: KDA itself
+ *                    ("Ten questions" Q8).  Same as kda_chunk_fwd / kda_decode_step.
+ *  KDA_GATE_SCALAR   gate = log_alpha [.., H] fp32, one decay per (token, head) shared by
+ *                    all channels: Gated DeltaNet ("22,580" §08).  The kernels apply the
+ *                    scalar to every channel with the arithmetic of KDA_GATE_CHANNEL, so
+ *                    the result is bit-identical to that form fed the broadcast gate.
+ *  KDA_GATE_NONE     gate = NULL, alpha = 1: DeltaNet ("22,580" §5-§6).
+ *  KDA_GATE_FUSED    gate = f [.., H, dk] in the input dtype, with A_log, dt_bias [H, dk]
+ *                    fp32: log_alpha = -exp(A_log) * softplus(f + dt_bias),
+ *                    softplus(x) = ln(1 + e^x) -- the gate line read out in "Ten questions"
+ *                    Q9, computed in the kernel in fp32, so the log_alpha stream (4 bytes
+ *                    per channel) becomes f in the input dtype.  log_alpha is kept >= -1e4
+ *                    (alpha = e^-1e4 is 0 in fp32 either way).
+ * Flags (any combination; 0 = none):
+ *  KDA_NORM_Q, KDA_NORM_K  q (resp. k) is scaled to unit L2 length per (token, head) in the
+ *                    kernel, x / max(||x||_2, 1e-12), fp32 ("22,580" §5.2 layer code).
+ *  KDA_BETA_LOGIT    beta holds logits: beta_t = 1 / (1 + e^-b_t) ("Ten questions" Q9).
+ * A_log and dt_bias are used (and must be non-NULL) only with KDA_GATE_FUSED.
+ */
+enum kda_gate_kind {
+    KDA_GATE_CHANNEL = 0,
+    KDA_GATE_SCALAR = 1,
+    KDA_GATE_NONE = 2,
+    KDA_GATE_FUSED = 3
+};
+enum kda_gate_flags { KDA_NORM_Q = 1, KDA_NORM_K = 2, KDA_BETA_LOGIT = 4 };
+
+/*
+ * kda_chunk_fwd_ex -- kda_chunk_fwd with a gate form and flags (above).
+ * Layouts, sizes, workspace, results and errors are those of kda_chunk_fwd, with
+ * log_alpha replaced by (gate_kind, gate, A_log, dt_bias, flags):
+ *   gate     CHANNEL: [T_total, H, dk] fp32;  SCALAR: [T_total, H] fp32;  NONE: NULL;
+ *            FUSED: f [T_total, H, dk] dtype
+ *   A_log, dt_bias  FUSED only: [H, dk] fp32 each
+ *   beta     [T_total, H] fp32: beta itself, or logits with KDA_BETA_LOGIT
+ * Errors as kda_chunk_fwd, plus KDA_ERR_GATE (unknown gate_kind or flags, gate NULL for a
+ * form that needs it or non-NULL for KDA_GATE_NONE, A_log or dt_bias NULL for KDA_GATE_FUSED).
+ */
+int kda_chunk_fwd_ex(const void *q, const void *k, const void *v, int gate_kind, const void *gate,
+                     const float *A_log, const float *dt_bias, int flags, const float *beta,
+                     const float *S0, const int32_t *cu_seqlens, void *out, float *S_final, int B,
+                     int T, int H, int dk, int dv, int C, int dtype, kda_stream_t stream);
+
+/*
+ * kda_chunk_bwd -- gradients of a prefill: the backward pass for training.
+ * The pages discuss training ("22,580" §6.1: the chunked prefill is the training-time path)
+ * but print no backward pass; this is the reverse-mode derivative of the chunked algorithm
+ * of kda_chunk_fwd ("22,580" §6.3 with the decay of §08/§9.1), recomputing the forward's
+ * chunk states itself.  For L = sum(dO * o) + sum(dS_final * S_final) it returns dL/d of
+ * every input.  fp32 arithmetic (the products are not on the tensor cores).
+ *   q, k, v, gate_kind, gate, beta, S0, cu_seqlens, B, T, H, dk, dv, C, dtype: as
+ *            kda_chunk_fwd_ex, with gate_kind KDA_GATE_CHANNEL, KDA_GATE_SCALAR or
+ *            KDA_GATE_NONE and no flags (the fused gate is not differentiated here)
+ *   dO       [T_total, H, dv]  dtype      gradient of o
+ *   dS_final [N, H, dk, dv]    fp32 or NULL (zero)
+ *   dq, dk   [T_total, H, dk]  dtype      written
+ *   dv       [T_total, H, dv]  dtype      written
+ *   dgate    CHANNEL: dlog_alpha [T_total, H, dk] fp32; SCALAR: [T_total, H] fp32 (the sum
+ *            over channels); NONE: ignored (may be NULL)
+ *   dbeta    [T_total, H]      fp32       written
+ *   dS0      [N, H, dk, dv]    fp32 or NULL (not written)
+ * Workspace: taken with cudaMallocAsync on `stream` from the default pool and freed on it:
+ * one fp32 state checkpoint per 16-token chunk per (head, 64-column d_v half) -- dk * dv * 4
+ * bytes per 16 tokens per head -- plus (3 dk + 1) * 4 bytes per token-head per d_v half.
+ * Errors: as kda_chunk_fwd_ex (KDA_ERR_GATE for the fused form or any flag), KDA_ERR_NULL for
+ * dO, dq, dk, dv, dbeta (or dgate with a decay form) NULL while T_total > 0, KDA_ERR_ALIAS
+ * for an output overlapping an input or another output.
+ */
+int kda_chunk_bwd(const void *q, const void *k, const void *v, int gate_kind, const void *gate,
+                  const float *beta, const float *S0, const int32_t *cu_seqlens, const void *dO,
+                  const float *dS_final, void *dq, void *dk, void *dv, float *dgate, float *dbeta,
+                  float *dS0, int B, int T, int H, int dk_, int dv_, int C, int dtype,
+                  kda_stream_t stream);
 
 /*
  * kda_decode_step -- one recurrent step (one new token) for N independent sequences.
@@ -158,11 +240,44 @@ int kda_decode_step(const void *q, const void *k, const void *v, const float *lo
                     int dv, int dtype, kda_stream_t stream);
 
 /*
+ * kda_decode_ex -- decode from an indexed state pool, L new tokens per sequence.
+ * For each sequence n < N with idx = state_idx[n] (or n when state_idx is NULL), the
+ * recurrence (in the gate form given, with flags, as in kda_chunk_fwd_ex) runs over the
+ * sequence's L new tokens in order from state_pool[idx], writes o for each token and
+ * stores the state back to state_pool[idx] once, after the last token.  This is the step of
+ * a serving cache ("Ten questions" Q10: the state is a fixed 16,384-cell board per head
+ * whatever the context length) and of multi-token (speculative) steps: one call over L
+ * tokens gives exactly the results of L calls with one token each.
+ *   q, k          [N, L, H, dk]     dtype
+ *   v             [N, L, H, dv]     dtype
+ *   gate          per gate_kind: [N, L, H, dk] fp32 / [N, L, H] fp32 / NULL / f [N, L, H, dk] dtype
+ *   A_log, dt_bias  [H, dk] fp32 (KDA_GATE_FUSED only)
+ *   beta          [N, L, H]         fp32 (logits with KDA_BETA_LOGIT)
+ *   state_pool    [P, H, dk, dv]    fp32, read and updated in place
+ *   state_idx     [N] int32 or NULL: the pool slot of each sequence.  A negative entry
+ *                 skips its sequence (nothing read or written, out untouched: padding).
+ *                 Entries must be distinct (two sequences on one slot race).  An entry >= P
+ *                 is skipped too and recorded: the next kda_device_status() returns
+ *                 KDA_ERR_INDEX.  NULL means slot n for sequence n and requires P >= N.
+ *   out           [N, L, H, dv]     dtype
+ * Memory-bound: each selected state is read once and written once per call.
+ * Errors: KDA_ERR_NULL, KDA_ERR_DIM (N, H, L, P < 1, dk or dv not in {32, 64, 128}, P < N
+ * without state_idx), KDA_ERR_DTYPE, KDA_ERR_ALIGN, KDA_ERR_ALIAS (out or state_pool
+ * overlapping an input or each other), KDA_ERR_GATE, KDA_ERR_CUDA.
+ */
+int kda_decode_ex(const void *q, const void *k, const void *v, int gate_kind, const void *gate,
+                  const float *A_log, const float *dt_bias, int flags, const float *beta,
+                  float *state_pool, const int32_t *state_idx, void *out, int N, int L, int H,
+                  int dk, int dv, int P, int dtype, kda_stream_t stream);
+
+/*
  * kda_device_status -- synchronises the current device, then reports whether any
  * libkda kernel since the previous call gave up one of its bounded device-side
  * waits (tensor-core completion barriers; each waits at most about two seconds
- * and then abandons its work item instead of hanging).  Clears that record.
- * Returns KDA_OK, KDA_ERR_TIMEOUT, or KDA_ERR_CUDA (the synchronisation failed).
+ * and then abandons its work item instead of hanging), or skipped a kda_decode_ex
+ * sequence whose state index was >= the pool size.  Clears that record.
+ * Returns KDA_OK, KDA_ERR_TIMEOUT (a wait gave up; reported first), KDA_ERR_INDEX, or
+ * KDA_ERR_CUDA (the synchronisation failed).
  */
 int kda_device_status(void);
 

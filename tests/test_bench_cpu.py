@@ -143,3 +143,47 @@ def test_prefill_parity_pairs_index_the_packed_token_axis():
     out4 = torch.randn(2, 7, 3, 32)                    # the [B, T, H, dv] view of a fixed-length call
     o, _ = bench.prefill_pairs(out4, torch.zeros(2, 3, 32, 32), fixed)(1, 2)
     np.testing.assert_array_equal(o, out4[1, :, 2].numpy())
+
+
+def test_decode_variant_oracle_replays_each_sequences_tokens_in_order():
+    """cpu_baseline_decode_ex packs, per sequence, the L tokens of every call in call order and
+    starts from that sequence's state; checked against the oracle run by hand on one pair."""
+    sys.path.insert(0, ROOT)
+    import numpy as np
+    import bench
+    import oracle
+    from gated_delta_rule_119_b200.inputs import make_decode_state, make_form_inputs
+    oracle.build()
+    N, L, H, d = 3, 2, 2, 32
+    ins = [make_form_inputs(N, L, H, d, d, "f32", (9, c), "fused", raw=True) for c in range(2)]
+    S0 = make_decode_state(N, H, d, d, 9)
+    n, h = 2, 1
+    views = [bench.oracle_view(i) for i in ins]
+    pick = lambda name: np.concatenate([np.asarray(getattr(v, name))[n * L:(n + 1) * L, h:h + 1]
+                                        for v in views])
+    ro, rs = oracle.recurrent_full(pick("q"), pick("k"), pick("v"), pick("log_alpha"), pick("beta"),
+                                   S0[n:n + 1, h:h + 1].copy())
+    cb = bench.cpu_baseline_decode_ex(ins, S0, L, 0.05, lambda a, b: (ro[:, 0], rs[0, 0]))
+    assert cb["kind"] == "oracle" and cb["value"] > 0 and "parity" in cb
+    # the function's packing of that pair equals the hand-built token stream
+    outs, states = oracle.recurrent(*[np.stack([np.asarray(getattr(v, x)).reshape(N, L, *np.shape(getattr(v, x))[1:])
+                                                for v in views], 1).reshape(N * 2 * L, *np.shape(getattr(views[0], x))[1:])
+                                      for x in ("q", "k", "v", "log_alpha", "beta")],
+                                    S0, np.arange(N + 1) * 2 * L, tasks=[(n, h)])
+    np.testing.assert_allclose(outs[0], ro[:, 0], rtol=0, atol=0)
+    np.testing.assert_allclose(states[0], rs[0, 0], rtol=0, atol=0)
+
+
+def test_oracle_view_applies_the_gate_front_end():
+    sys.path.insert(0, ROOT)
+    import numpy as np
+    import bench
+    from oracle import gates
+    from gated_delta_rule_119_b200.inputs import make_form_inputs
+    inp = make_form_inputs(2, 20, 2, 32, 32, "bf16", 10, "fused", raw=True)
+    v = bench.oracle_view(inp)
+    np.testing.assert_array_equal(v.log_alpha, gates.fused_log_alpha(inp.f, inp.A_log, inp.dt_bias))
+    np.testing.assert_allclose(np.linalg.norm(v.k, axis=-1), 1.0, rtol=1e-14)
+    np.testing.assert_array_equal(v.beta, gates.sigmoid(inp.beta))
+    s = make_form_inputs(2, 20, 2, 32, 32, "f32", 11, "scalar")
+    assert bench.oracle_view(s).log_alpha.shape == (40, 2, 32)

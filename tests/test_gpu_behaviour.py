@@ -39,9 +39,17 @@ def test_side_stream_gives_the_default_stream_result():
     assert kda_device_status() == 0
 
 
-@pytest.mark.parametrize("gates", ["default", "extremes"])
+@pytest.mark.parametrize("gates", ["default", "extremes", "clear"])
 def test_tensor_core_path_is_deterministic(gates):
-    inp = make_inputs(2, 1000, 4, 128, 128, "bf16", 1202, state=True, gates=gates)
+    """Three calls give bit-identical results.  "clear" puts log_alpha = -1e4 on whole heads
+    and on scattered tokens, so that blocks take the exact per-channel path (decay spread
+    beyond the rescaled factors' range) beside the fast and the block paths."""
+    inp = make_inputs(2, 1000, 4, 128, 128, "bf16", 1202, state=True,
+                      gates="default" if gates == "clear" else gates)
+    if gates == "clear":
+        inp.log_alpha[:, 0] = -1e4
+        inp.log_alpha[::5, 1, ::3] = -1e4
+        inp.log_alpha[3::11, 2] = -1e4
     d = to_torch(inp)
     outs = [call(d) for _ in range(3)]
     torch.cuda.synchronize()
@@ -149,3 +157,25 @@ def test_concurrent_host_threads_match_sequential_calls():
             assert torch.equal(o, o_ref) and torch.equal(s, s_ref)
     from gated_delta_rule_119_b200 import kda_device_status
     assert kda_device_status() == 0
+
+
+def test_malformed_cu_seqlens_stay_in_bounds():
+    """Offsets that are not non-decreasing ([0, T, 0, T]: two clamped sequences of T tokens
+    over the same tokens) ask for more workspace slots than the call holds; the slot table
+    caps them, so the call completes without a device error.  Results of such a call are
+    unspecified except that the first sequence, whose slots come first, is still exact."""
+    T, H = 2048, 2
+    inp = make_inputs(1, T, H, 128, 128, "bf16", 1290, state=True)
+    from gated_delta_rule_119_b200 import kda_chunk_fwd, kda_device_status
+    d = to_torch(inp)
+    packed = {k_: d[k_].reshape(T, *d[k_].shape[2:]) for k_ in ("q", "k", "v", "log_alpha", "beta")}
+    cu = torch.tensor([0, T, 0, T], dtype=torch.int32, device="cuda")
+    S0 = torch.cat([d["S0"]] * 3)
+    o, S = kda_chunk_fwd(packed["q"], packed["k"], packed["v"], packed["log_alpha"],
+                         packed["beta"], S0, cu)
+    torch.cuda.synchronize()
+    assert kda_device_status() == 0
+    _, rs = oracle.recurrent_full(inp.q, inp.k, inp.v, inp.log_alpha, inp.beta, inp.S0,
+                                  inp.offsets())
+    assert rel_err(S[0].cpu().numpy(), rs[0]) <= TOL["bf16"]
+    np.testing.assert_array_equal(S[1].cpu().numpy(), inp.S0[0])     # the empty sequence

@@ -144,6 +144,20 @@ def test_degenerate_gates(dtype):
 
 
 @pytest.mark.parametrize("dtype", ["f32", "bf16"])
+def test_block_spread_past_fp32_normal_range(dtype):
+    """Channels whose decay over 16 rows sums to about 90-135 (past fp32's normal range, e^-87,
+    for an unscaled running product; short of the exact path's limit of 140) beside weakly
+    decaying channels in the same heads: the block path's rescaled factors must keep their
+    precision on every row, the last rows of each 16-row block included."""
+    inp = make_inputs(2, 300, 3, 128, 128, dtype, 23, state=True)
+    rng = np.random.default_rng(24)
+    inp.log_alpha[:, 0, :32] = rng.uniform(-8.4, -5.6, size=(inp.total_tokens, 32)).astype(np.float32)
+    inp.log_alpha[:, 1, ::4] = -7.0
+    inp.log_alpha[:, 2, 64:] = rng.uniform(-6.5, -6.0, size=(inp.total_tokens, 64)).astype(np.float32)
+    check_against_oracle(inp)
+
+
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
 def test_extreme_gates_small(dtype):
     check_against_oracle(make_inputs(2, 300, 4, 128, 128, dtype, 19, gates="extremes",
                                      state=True))
