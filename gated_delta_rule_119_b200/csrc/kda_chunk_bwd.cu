@@ -36,9 +36,10 @@ constexpr int kThreads = 256;
 constexpr int kC = 16;
 static_assert(kThreads == 16 * kC, "the K / P and gradient passes map thread t to (row or column t / 16, channel group t % 16)");
 
+// Row pitches are padded to a multiple of 4 floats so that rows can be read 16 bytes at a time.
 template <int DK, int DVH>
 struct BwdLayout {
-    static constexpr int LK = DK + 1, LV = DVH + 1, LC = kC + 1;
+    static constexpr int LK = DK + 4, LV = DVH + 4, LC = kC + 1;
     // [kC][LK] arrays
     static constexpr int Q = 0, Kk = Q + kC * LK, AL = Kk + kC * LK, GA = AL + kC * LK, KA = GA + kC * LK,
                          KG = KA + kC * LK, SQ = KG + kC * LK, KK = SQ + kC * LK, DQ = KK + kC * LK,
@@ -52,7 +53,8 @@ struct BwdLayout {
     static constexpr int KM = DR + kC * LV, TM = KM + kC * LC, PM = TM + kC * LC, DPM = PM + kC * LC,
                          DTM = DPM + kC * LC, XM = DTM + kC * LC;
     static constexpr int GC = XM + kC * LC, BT = GC + DK, DB = BT + kC, DGC = DB + kC;
-    static constexpr int floats = DGC + DK;
+    static constexpr int DGP = DGC + DK;      // [kThreads / DK][DK] partial last-row g terms
+    static constexpr int floats = DGP + kThreads;
     static constexpr size_t bytes = (size_t)floats * sizeof(float);
 };
 
@@ -73,10 +75,21 @@ __device__ __forceinline__ size_t part_index(const BwdArgs &b, int split, size_t
     return ((size_t)split * b.a.T_total * b.a.H + th) * (3 * (size_t)dk + 1);
 }
 
+__device__ __forceinline__ float4 ld4(const float *p) { return *reinterpret_cast<const float4 *>(p); }
+
+// acc += a . b over four consecutive k, in k order.
+__device__ __forceinline__ float dot4(float4 a, float4 b, float acc) {
+    return fmaf(a.w, b.w, fmaf(a.z, b.z, fmaf(a.y, b.y, fmaf(a.x, b.x, acc))));
+}
+
 template <typename Tin, int DK, int DVH>
 __global__ void __launch_bounds__(kThreads, 1) kda_chunk_bwd_kernel(BwdArgs b) {
     using L = BwdLayout<DK, DVH>;
     constexpr int LK = L::LK, LV = L::LV, LC = L::LC, CH = kC;
+    constexpr int RPT = kC * DVH / kThreads;   // rows per thread of the [C][dv] products
+    constexpr int CPT = DK * DVH / kThreads;   // rows per thread of the [dk][dv] products
+    constexpr int R7 = kC * DK / kThreads;     // rows per thread of the [C][dk] products
+    static_assert(RPT >= 1 && CPT % 4 == 0 && R7 >= 1 && DK % 4 == 0 && DVH % 4 == 0, "backward tiling");
     extern __shared__ float sm[];
     float *Q = sm + L::Q, *Kk = sm + L::Kk, *AL = sm + L::AL, *GA = sm + L::GA, *KA = sm + L::KA;
     float *KG = sm + L::KG, *SQ = sm + L::SQ, *KK = sm + L::KK, *DQ = sm + L::DQ, *DKc = sm + L::DKc;
@@ -84,6 +97,7 @@ __global__ void __launch_bounds__(kThreads, 1) kda_chunk_bwd_kernel(BwdArgs b) {
     float *U = sm + L::U, *DO = sm + L::DO, *DU = sm + L::DU, *DR = sm + L::DR;
     float *KM = sm + L::KM, *TM = sm + L::TM, *PM = sm + L::PM, *DPM = sm + L::DPM, *DTM = sm + L::DTM;
     float *XM = sm + L::XM, *GC = sm + L::GC, *BT = sm + L::BT, *DB = sm + L::DB, *DGC = sm + L::DGC;
+    float *DGP = sm + L::DGP;
 
     const KdaChunkArgs &a = b.a;
     const int H = a.H, dv = a.dv;
@@ -216,19 +230,31 @@ __global__ void __launch_bounds__(kThreads, 1) kda_chunk_bwd_kernel(BwdArgs b) {
             }
         }
         __syncthreads();
-        // r = v - (k gamma) S;  then u = T Diag(beta) r
-        for (int idx = tid; idx < CH * DVH; idx += kThreads) {
-            const int r = idx / DVH, j = idx % DVH;
-            float acc = V[r * LV + j];
-            for (int c = 0; c < DK; ++c) acc = fmaf(-KG[r * LK + c], S[c * LV + j], acc);
-            R[r * LV + j] = acc;
-        }
-        __syncthreads();
-        for (int idx = tid; idx < CH * DVH; idx += kThreads) {
-            const int r = idx / DVH, j = idx % DVH;
-            float acc = 0.f;
-            for (int i = 0; i <= r; ++i) acc = fmaf(TM[r * LC + i] * BT[i], R[i * LV + j], acc);
-            U[r * LV + j] = acc;
+        // r = v - (k gamma) S;  then u = T Diag(beta) r.  Thread: column j, RPT rows.
+        {
+            const int j = tid % DVH, r0 = (tid / DVH) * RPT;
+            float acc[RPT];
+#pragma unroll
+            for (int t = 0; t < RPT; ++t) acc[t] = V[(r0 + t) * LV + j];
+            for (int c = 0; c < DK; c += 4) {
+                const float4 s4 = make_float4(S[c * LV + j], S[(c + 1) * LV + j], S[(c + 2) * LV + j],
+                                              S[(c + 3) * LV + j]);
+#pragma unroll
+                for (int t = 0; t < RPT; ++t) {
+                    const float4 kg = ld4(KG + (r0 + t) * LK + c);
+                    acc[t] = dot4(make_float4(-kg.x, -kg.y, -kg.z, -kg.w), s4, acc[t]);
+                }
+            }
+#pragma unroll
+            for (int t = 0; t < RPT; ++t) R[(r0 + t) * LV + j] = acc[t];
+            __syncthreads();
+#pragma unroll
+            for (int t = 0; t < RPT; ++t) {
+                const int r = r0 + t;
+                float u = 0.f;
+                for (int i = 0; i <= r; ++i) u = fmaf(TM[r * LC + i] * BT[i], R[i * LV + j], u);
+                U[r * LV + j] = u;
+            }
         }
         __syncthreads();
     };
@@ -240,12 +266,25 @@ __global__ void __launch_bounds__(kThreads, 1) kda_chunk_bwd_kernel(BwdArgs b) {
         float *dst = ckpt_block(ci);
         for (int idx = tid; idx < DK * DVH; idx += kThreads) dst[idx] = S[(idx / DVH) * LV + idx % DVH];
         chunk_terms(c0, nr, false);
-        // S <- Diag(gamma_last) S + (k kappa)^T u, element by element in place
-        for (int idx = tid; idx < DK * DVH; idx += kThreads) {
-            const int c = idx / DVH, j = idx % DVH;
-            float acc = GC[c] * S[c * LV + j];
-            for (int r = 0; r < CH; ++r) acc = fmaf(KK[r * LK + c], U[r * LV + j], acc);
-            S[c * LV + j] = acc;
+        // S <- Diag(gamma_last) S + (k kappa)^T u, in place.  Thread: column j, CPT rows.
+        {
+            const int j = tid % DVH, c0 = (tid / DVH) * CPT;
+            float acc[CPT];
+#pragma unroll
+            for (int t = 0; t < CPT; ++t) acc[t] = GC[c0 + t] * S[(c0 + t) * LV + j];
+            for (int r = 0; r < CH; ++r) {
+                const float u = U[r * LV + j];
+#pragma unroll
+                for (int t = 0; t < CPT; t += 4) {
+                    const float4 kk = ld4(KK + r * LK + c0 + t);
+                    acc[t] = fmaf(kk.x, u, acc[t]);
+                    acc[t + 1] = fmaf(kk.y, u, acc[t + 1]);
+                    acc[t + 2] = fmaf(kk.z, u, acc[t + 2]);
+                    acc[t + 3] = fmaf(kk.w, u, acc[t + 3]);
+                }
+            }
+#pragma unroll
+            for (int t = 0; t < CPT; ++t) S[(c0 + t) * LV + j] = acc[t];
         }
         __syncthreads();
     }
@@ -263,58 +302,82 @@ __global__ void __launch_bounds__(kThreads, 1) kda_chunk_bwd_kernel(BwdArgs b) {
         __syncthreads();
         chunk_terms(c0, nr, true);
 
-        // du = P^T dO + (k kappa) dS'
-        for (int idx = tid; idx < CH * DVH; idx += kThreads) {
-            const int i = idx / DVH, j = idx % DVH;
-            float acc = 0.f;
-            for (int r = i; r < CH; ++r) acc = fmaf(PM[r * LC + i], DO[r * LV + j], acc);
-            for (int c = 0; c < DK; ++c) acc = fmaf(KK[i * LK + c], DS[c * LV + j], acc);
-            DU[i * LV + j] = acc;
-        }
-        __syncthreads();
-        // dr = Diag(beta) T^T du (this half's dv rows)
-        for (int idx = tid; idx < CH * DVH; idx += kThreads) {
-            const int i = idx / DVH, j = idx % DVH;
-            float acc = 0.f;
-            for (int r = i; r < CH; ++r) acc = fmaf(TM[r * LC + i], DU[r * LV + j], acc);
-            acc *= BT[i];
-            DR[i * LV + j] = acc;
-            if (i < nr) dvg[((size_t)(c0 + i) * H + h) * dv + j0 + j] = kda::from_f32<Tin>(acc);
+        // du = P^T dO + (k kappa) dS', then dr = Diag(beta) T^T du (this half's dv rows).
+        // Thread: column j, RPT rows.
+        {
+            const int j = tid % DVH, i0 = (tid / DVH) * RPT;
+            float acc[RPT];
+#pragma unroll
+            for (int t = 0; t < RPT; ++t) {
+                const int i = i0 + t;
+                float a0 = 0.f;
+                for (int r = i; r < CH; ++r) a0 = fmaf(PM[r * LC + i], DO[r * LV + j], a0);
+                acc[t] = a0;
+            }
+            for (int c = 0; c < DK; c += 4) {
+                const float4 d4 = make_float4(DS[c * LV + j], DS[(c + 1) * LV + j], DS[(c + 2) * LV + j],
+                                              DS[(c + 3) * LV + j]);
+#pragma unroll
+                for (int t = 0; t < RPT; ++t) acc[t] = dot4(ld4(KK + (i0 + t) * LK + c), d4, acc[t]);
+            }
+#pragma unroll
+            for (int t = 0; t < RPT; ++t) DU[(i0 + t) * LV + j] = acc[t];
+            __syncthreads();
+#pragma unroll
+            for (int t = 0; t < RPT; ++t) {
+                const int i = i0 + t;
+                float a1 = 0.f;
+                for (int r = i; r < CH; ++r) a1 = fmaf(TM[r * LC + i], DU[r * LV + j], a1);
+                a1 *= BT[i];
+                DR[i * LV + j] = a1;
+                if (i < nr) dvg[((size_t)(c0 + i) * H + h) * dv + j0 + j] = kda::from_f32<Tin>(a1);
+            }
         }
         // dP = tril(dO u^T) and dT' = tril(du r^T) over this half's columns
         for (int idx = tid; idx < CH * CH; idx += kThreads) {
             const int r = idx / CH, i = idx % CH;
             float p = 0.f, t = 0.f;
             if (i <= r) {
-                for (int j = 0; j < DVH; ++j) {
-                    p = fmaf(DO[r * LV + j], U[i * LV + j], p);
-                    t = fmaf(DU[r * LV + j], R[i * LV + j], t);
+                for (int j = 0; j < DVH; j += 4) {
+                    p = dot4(ld4(DO + r * LV + j), ld4(U + i * LV + j), p);
+                    t = dot4(ld4(DU + r * LV + j), ld4(R + i * LV + j), t);
                 }
             }
             DPM[r * LC + i] = p;
             DTM[r * LC + i] = t;
         }
         __syncthreads();
-        // the decay-weighted elementwise terms, one thread per channel:
-        //   d(s q gamma) = dO S^T, d(k gamma) = -dr S^T, d(k kappa) = u dS'^T, d gamma_last
-        for (int c = tid; c < DK; c += kThreads) {
+        // the decay-weighted elementwise terms: d(s q gamma) = dO S^T, d(k gamma) = -dr S^T,
+        // d(k kappa) = u dS'^T, and the last row's g terms.  Thread: channel c, R7 rows.
+        {
+            const int c = tid % DK, g7 = tid / DK, r0 = g7 * R7;
+            float dsq[R7], dkg[R7], dkk[R7];
+#pragma unroll
+            for (int t = 0; t < R7; ++t) dsq[t] = dkg[t] = dkk[t] = 0.f;
             float gl = 0.f;
-            for (int j = 0; j < DVH; ++j) gl = fmaf(DS[c * LV + j], S[c * LV + j], gl);
-            float kkp = 0.f;
-            for (int r = 0; r < CH; ++r) {
-                float dsq = 0.f, dkg = 0.f, dkk = 0.f;
-                for (int j = 0; j < DVH; ++j) {
-                    const float s = S[c * LV + j];
-                    dsq = fmaf(DO[r * LV + j], s, dsq);
-                    dkg = fmaf(-DR[r * LV + j], s, dkg);
-                    dkk = fmaf(U[r * LV + j], DS[c * LV + j], dkk);
+            for (int j = 0; j < DVH; j += 4) {
+                const float4 s4 = ld4(S + c * LV + j), d4 = ld4(DS + c * LV + j);
+                if (g7 == 0) gl = dot4(d4, s4, gl);
+#pragma unroll
+                for (int t = 0; t < R7; ++t) {
+                    const int r = r0 + t;
+                    const float4 dr = ld4(DR + r * LV + j);
+                    dsq[t] = dot4(ld4(DO + r * LV + j), s4, dsq[t]);
+                    dkg[t] = dot4(make_float4(-dr.x, -dr.y, -dr.z, -dr.w), s4, dkg[t]);
+                    dkk[t] = dot4(ld4(U + r * LV + j), d4, dkk[t]);
                 }
-                DQ[r * LK + c] = scale * GA[r * LK + c] * dsq;
-                DKc[r * LK + c] = GA[r * LK + c] * dkg + KA[r * LK + c] * dkk;
-                DG[r * LK + c] = dsq * SQ[r * LK + c] + dkg * KG[r * LK + c] - dkk * KK[r * LK + c];
-                kkp = fmaf(dkk, KK[r * LK + c], kkp);
             }
-            DGC[c] = GC[c] * gl + kkp;          // both go to the last row's g
+            float kkp = 0.f;
+#pragma unroll
+            for (int t = 0; t < R7; ++t) {
+                const int r = r0 + t;
+                DQ[r * LK + c] = scale * GA[r * LK + c] * dsq[t];
+                DKc[r * LK + c] = GA[r * LK + c] * dkg[t] + KA[r * LK + c] * dkk[t];
+                DG[r * LK + c] = dsq[t] * SQ[r * LK + c] + dkg[t] * KG[r * LK + c] - dkk[t] * KK[r * LK + c];
+                kkp = fmaf(dkk[t], KK[r * LK + c], kkp);
+            }
+            DGP[g7 * DK + c] = kkp;
+            if (g7 == 0) DGC[c] = GC[c] * gl;   // the partial terms are added below, in group order
         }
         // dbeta from T' = T Diag(beta); dT = dT' Diag(beta); X = dT T^T
         if (tid < CH) {
@@ -324,6 +387,11 @@ __global__ void __launch_bounds__(kThreads, 1) kda_chunk_bwd_kernel(BwdArgs b) {
             DB[i] = acc;
         }
         __syncthreads();
+        for (int c = tid; c < DK; c += kThreads) {
+            float acc = DGC[c];
+            for (int g = 0; g < kThreads / DK; ++g) acc += DGP[g * DK + c];
+            DGC[c] = acc;                     // both go to the last row's g
+        }
         for (int idx = tid; idx < CH * CH; idx += kThreads) {
             const int r = idx / CH, m = idx % CH;
             float acc = 0.f;
@@ -399,13 +467,26 @@ __global__ void __launch_bounds__(kThreads, 1) kda_chunk_bwd_kernel(BwdArgs b) {
             }
         }
         if (tid < nr) b.part[part_index(b, split, (size_t)(c0 + tid) * H + h, DK) + 3 * DK] = DB[tid];
-        // dS for the previous chunk, in place: (s q gamma)^T dO + Diag(gamma_last) dS' - (k gamma)^T dr
-        for (int idx = tid; idx < DK * DVH; idx += kThreads) {
-            const int c = idx / DVH, j = idx % DVH;
-            float acc = GC[c] * DS[c * LV + j];
-            for (int r = 0; r < CH; ++r)
-                acc = fmaf(SQ[r * LK + c], DO[r * LV + j], fmaf(-KG[r * LK + c], DR[r * LV + j], acc));
-            DS[c * LV + j] = acc;
+        // dS for the previous chunk, in place: (s q gamma)^T dO + Diag(gamma_last) dS' - (k gamma)^T dr.
+        // Thread: column j, CPT rows.
+        {
+            const int j = tid % DVH, cb = (tid / DVH) * CPT;
+            float acc[CPT];
+#pragma unroll
+            for (int t = 0; t < CPT; ++t) acc[t] = GC[cb + t] * DS[(cb + t) * LV + j];
+            for (int r = 0; r < CH; ++r) {
+                const float d = DO[r * LV + j], e = DR[r * LV + j];
+#pragma unroll
+                for (int t = 0; t < CPT; t += 4) {
+                    const float4 sq = ld4(SQ + r * LK + cb + t), kg = ld4(KG + r * LK + cb + t);
+                    acc[t] = fmaf(sq.x, d, fmaf(-kg.x, e, acc[t]));
+                    acc[t + 1] = fmaf(sq.y, d, fmaf(-kg.y, e, acc[t + 1]));
+                    acc[t + 2] = fmaf(sq.z, d, fmaf(-kg.z, e, acc[t + 2]));
+                    acc[t + 3] = fmaf(sq.w, d, fmaf(-kg.w, e, acc[t + 3]));
+                }
+            }
+#pragma unroll
+            for (int t = 0; t < CPT; ++t) DS[(cb + t) * LV + j] = acc[t];
         }
         __syncthreads();
     }

@@ -351,9 +351,10 @@ __global__ void __launch_bounds__(NTHR, 2)
     const int c2 = 2 * (tid & 63), eb = tid >> 6;
     float2 la[16];
     uint32_t kr2[16];
-    float2 alog = make_float2(0.f, 0.f), dtb = make_float2(0.f, 0.f);
+    float2 eA = make_float2(0.f, 0.f), dtb = make_float2(0.f, 0.f);   // e^A_log, dt_bias of the two channels
     if (GATE == kda::GATE_FUSED) {
-        alog = *reinterpret_cast<const float2 *>(a.A_log + (size_t)h * DK + c2);
+        const float2 alog = *reinterpret_cast<const float2 *>(a.A_log + (size_t)h * DK + c2);
+        eA = make_float2(expf(alog.x), expf(alog.y));
         dtb = *reinterpret_cast<const float2 *>(a.dt_bias + (size_t)h * DK + c2);
     }
 #pragma unroll
@@ -364,7 +365,7 @@ __global__ void __launch_bounds__(NTHR, 2)
             la[rr] = ok ? *reinterpret_cast<const float2 *>(sKQ + 4 * (r * DK + c2)) : make_float2(0.f, 0.f);
         } else if (GATE == kda::GATE_FUSED) {
             const float2 f = unpack_bf16(*reinterpret_cast<const uint32_t *>(sKQ + 2 * (r * DK + c2)));
-            la[rr] = ok ? make_float2(kda::fused_log_alpha(f.x, alog.x, dtb.x), kda::fused_log_alpha(f.y, alog.y, dtb.y))
+            la[rr] = ok ? make_float2(kda::fused_log_alpha_e(f.x, eA.x, dtb.x), kda::fused_log_alpha_e(f.y, eA.y, dtb.y))
                         : make_float2(0.f, 0.f);
         } else if (GATE == kda::GATE_SCALAR) {
             la[rr] = make_float2(sLa[r], sLa[r]);
