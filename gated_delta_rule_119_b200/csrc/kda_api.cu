@@ -2,6 +2,8 @@
 #include <stdio.h>
 #include <string.h>
 
+#include <atomic>
+
 #include "../../include/kda.h"
 #include "kda_common.cuh"
 
@@ -25,7 +27,25 @@ struct Span {
 Span span(const void *p, size_t bytes) { return {(uintptr_t)p, (uintptr_t)p + bytes}; }
 bool overlap(Span a, Span b) { return a.lo < b.hi && b.lo < a.hi && a.lo != a.hi && b.lo != b.hi; }
 
+constexpr int kMaxDevices = 64;
+// Per-device "already done" flags: only a shortcut, the set-up call is idempotent, so two host
+// threads that both find a flag clear both make it, which is harmless.
+std::atomic<bool> g_pool_configured[kMaxDevices] = {};
+
 }  // namespace
+
+cudaError_t kda_keep_pool_memory(int dev) {
+    if (dev >= 0 && dev < kMaxDevices && g_pool_configured[dev].load(std::memory_order_acquire))
+        return cudaSuccess;
+    cudaMemPool_t pool;
+    cudaError_t e = cudaDeviceGetDefaultMemPool(&pool, dev);
+    if (e != cudaSuccess) return e;
+    uint64_t keep = ~0ull;
+    e = cudaMemPoolSetAttribute(pool, cudaMemPoolAttrReleaseThreshold, &keep);
+    if (e != cudaSuccess) return e;
+    if (dev >= 0 && dev < kMaxDevices) g_pool_configured[dev].store(true, std::memory_order_release);
+    return cudaSuccess;
+}
 
 extern "C" const char *kda_status_string(int status) {
     switch (status) {
@@ -210,6 +230,7 @@ extern "C" int kda_chunk_bwd(const void *q, const void *k, const void *v, int ga
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return cuda_status(e);
+    if ((e = kda_keep_pool_memory(dev)) != cudaSuccess) return cuda_status(e);
     void *ws = nullptr;
     if ((e = cudaMallocAsync(&ws, kda_chunk_bwd_workspace_bytes(a), st)) != cudaSuccess) return cuda_status(e);
     e = kda_launch_chunk_bwd(a, dtype, dO, dS_final, dq, dk, dv, dgate, dbeta, dS0, ws, st);

@@ -32,9 +32,9 @@
 
 namespace {
 
-constexpr int kThreads = 256;
+constexpr int kThreads = 512;
 constexpr int kC = 16;
-static_assert(kThreads == 16 * kC, "the K / P and gradient passes map thread t to (row or column t / 16, channel group t % 16)");
+static_assert(kThreads == 32 * kC, "the K / P and gradient passes map warp w to row or column w, lane to a channel group");
 
 // Row pitches are padded to a multiple of 4 floats so that rows can be read 16 bytes at a time.
 template <int DK, int DVH>
@@ -83,13 +83,14 @@ __device__ __forceinline__ float dot4(float4 a, float4 b, float acc) {
 }
 
 template <typename Tin, int DK, int DVH>
-__global__ void __launch_bounds__(kThreads, 1) kda_chunk_bwd_kernel(BwdArgs b) {
+__global__ void __launch_bounds__(kThreads, 1) kda_chunk_bwd_kernel(BwdArgs b) {   // 16 warps, <= 128 registers
     using L = BwdLayout<DK, DVH>;
     constexpr int LK = L::LK, LV = L::LV, LC = L::LC, CH = kC;
     constexpr int RPT = kC * DVH / kThreads;   // rows per thread of the [C][dv] products
     constexpr int CPT = DK * DVH / kThreads;   // rows per thread of the [dk][dv] products
     constexpr int R7 = kC * DK / kThreads;     // rows per thread of the [C][dk] products
-    static_assert(RPT >= 1 && CPT % 4 == 0 && R7 >= 1 && DK % 4 == 0 && DVH % 4 == 0, "backward tiling");
+    static_assert(RPT >= 1 && (CPT % 4 == 0 || CPT < 4) && R7 >= 1 && DK % 32 == 0 && DVH % 4 == 0,
+                  "backward tiling");
     extern __shared__ float sm[];
     float *Q = sm + L::Q, *Kk = sm + L::Kk, *AL = sm + L::AL, *GA = sm + L::GA, *KA = sm + L::KA;
     float *KG = sm + L::KG, *SQ = sm + L::SQ, *KK = sm + L::KK, *DQ = sm + L::DQ, *DKc = sm + L::DKc;
@@ -182,13 +183,12 @@ __global__ void __launch_bounds__(kThreads, 1) kda_chunk_bwd_kernel(BwdArgs b) {
                 kp *= AL[r * LK + c];
             }
         }
-        // K and P: thread (i, channel group cg of 16) carries running products down the rows
-        // r >= i; the 16 groups of a column (lanes of one half-warp) are summed by shuffles.
-        // Every lane walks all CH rows (rows above i contribute zero) so that the full-warp
-        // shuffles are reached by all 32 lanes on every row.
+        // K and P: warp i, lane = channel group cg of 32, carries running products down the rows
+        // r >= i; the 32 groups of a column are summed by full-warp shuffles (every lane of the
+        // warp walks the same rows).
         {
-            const int i = tid >> 4, cg = tid & 15;
-            constexpr int CPT = DK / 16;
+            const int i = tid >> 5, cg = tid & 31;
+            constexpr int CPT = DK / 32;
             float f[CPT];
 #pragma unroll
             for (int m = 0; m < CPT; ++m) f[m] = 1.f;
@@ -197,7 +197,7 @@ __global__ void __launch_bounds__(kThreads, 1) kda_chunk_bwd_kernel(BwdArgs b) {
                 if (r >= i) {
 #pragma unroll
                     for (int m = 0; m < CPT; ++m) {
-                        const int c = cg + 16 * m;
+                        const int c = cg + 32 * m;
                         if (r > i) f[m] *= AL[r * LK + c];
                         const float kd = Kk[i * LK + c] * f[m];
                         sk = fmaf(Kk[r * LK + c], kd, sk);
@@ -205,7 +205,7 @@ __global__ void __launch_bounds__(kThreads, 1) kda_chunk_bwd_kernel(BwdArgs b) {
                     }
                 }
 #pragma unroll
-                for (int o = 8; o > 0; o >>= 1) {
+                for (int o = 16; o > 0; o >>= 1) {
                     sk += __shfl_xor_sync(0xffffffffu, sk, o);
                     sp += __shfl_xor_sync(0xffffffffu, sp, o);
                 }
@@ -274,13 +274,18 @@ __global__ void __launch_bounds__(kThreads, 1) kda_chunk_bwd_kernel(BwdArgs b) {
             for (int t = 0; t < CPT; ++t) acc[t] = GC[c0 + t] * S[(c0 + t) * LV + j];
             for (int r = 0; r < CH; ++r) {
                 const float u = U[r * LV + j];
+                if constexpr (CPT % 4 == 0) {
 #pragma unroll
-                for (int t = 0; t < CPT; t += 4) {
-                    const float4 kk = ld4(KK + r * LK + c0 + t);
-                    acc[t] = fmaf(kk.x, u, acc[t]);
-                    acc[t + 1] = fmaf(kk.y, u, acc[t + 1]);
-                    acc[t + 2] = fmaf(kk.z, u, acc[t + 2]);
-                    acc[t + 3] = fmaf(kk.w, u, acc[t + 3]);
+                    for (int t = 0; t < CPT; t += 4) {
+                        const float4 kk = ld4(KK + r * LK + c0 + t);
+                        acc[t] = fmaf(kk.x, u, acc[t]);
+                        acc[t + 1] = fmaf(kk.y, u, acc[t + 1]);
+                        acc[t + 2] = fmaf(kk.z, u, acc[t + 2]);
+                        acc[t + 3] = fmaf(kk.w, u, acc[t + 3]);
+                    }
+                } else {
+#pragma unroll
+                    for (int t = 0; t < CPT; ++t) acc[t] = fmaf(KK[r * LK + c0 + t], u, acc[t]);
                 }
             }
 #pragma unroll
@@ -420,14 +425,14 @@ __global__ void __launch_bounds__(kThreads, 1) kda_chunk_bwd_kernel(BwdArgs b) {
             DTM[r * LC + i] *= BT[r];            // dK
         }
         __syncthreads();
-        // through D = e^{g_r - g_i} in K and P: thread (x, channel group cg); as column i = x
+        // through D = e^{g_r - g_i} in K and P: warp x, lane = channel group cg; as column i = x
         // it walks rows r >= x, as row r = x it walks columns i <= x, each with running products.
         {
-            const int x = tid >> 4, cg = tid & 15;
-            constexpr int CPT = DK / 16;
+            const int x = tid >> 5, cg = tid & 31;
+            constexpr int CPT = DK / 32;
 #pragma unroll
             for (int m = 0; m < CPT; ++m) {
-                const int c = cg + 16 * m;
+                const int c = cg + 32 * m;
                 const float kx = Kk[x * LK + c], qx = Q[x * LK + c];
                 float f = 1.f, adk = 0.f, adg = 0.f;
                 for (int r = x; r < CH; ++r) {                    // x as the column i
@@ -476,13 +481,19 @@ __global__ void __launch_bounds__(kThreads, 1) kda_chunk_bwd_kernel(BwdArgs b) {
             for (int t = 0; t < CPT; ++t) acc[t] = GC[cb + t] * DS[(cb + t) * LV + j];
             for (int r = 0; r < CH; ++r) {
                 const float d = DO[r * LV + j], e = DR[r * LV + j];
+                if constexpr (CPT % 4 == 0) {
 #pragma unroll
-                for (int t = 0; t < CPT; t += 4) {
-                    const float4 sq = ld4(SQ + r * LK + cb + t), kg = ld4(KG + r * LK + cb + t);
-                    acc[t] = fmaf(sq.x, d, fmaf(-kg.x, e, acc[t]));
-                    acc[t + 1] = fmaf(sq.y, d, fmaf(-kg.y, e, acc[t + 1]));
-                    acc[t + 2] = fmaf(sq.z, d, fmaf(-kg.z, e, acc[t + 2]));
-                    acc[t + 3] = fmaf(sq.w, d, fmaf(-kg.w, e, acc[t + 3]));
+                    for (int t = 0; t < CPT; t += 4) {
+                        const float4 sq = ld4(SQ + r * LK + cb + t), kg = ld4(KG + r * LK + cb + t);
+                        acc[t] = fmaf(sq.x, d, fmaf(-kg.x, e, acc[t]));
+                        acc[t + 1] = fmaf(sq.y, d, fmaf(-kg.y, e, acc[t + 1]));
+                        acc[t + 2] = fmaf(sq.z, d, fmaf(-kg.z, e, acc[t + 2]));
+                        acc[t + 3] = fmaf(sq.w, d, fmaf(-kg.w, e, acc[t + 3]));
+                    }
+                } else {
+#pragma unroll
+                    for (int t = 0; t < CPT; ++t)
+                        acc[t] = fmaf(SQ[r * LK + cb + t], d, fmaf(-KG[r * LK + cb + t], e, acc[t]));
                 }
             }
 #pragma unroll

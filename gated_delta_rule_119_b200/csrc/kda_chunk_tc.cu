@@ -22,12 +22,13 @@
 // current chunk runs, one issues the tensor-core products, eight move the state, u and o
 // through tensor memory, and one stores o (TMA).
 //
-// Intra-chunk kernel, per (chunk, head):
-//  IN  one thread loads the chunk's log_alpha, k and q tiles by TMA into shared memory that
-//      later phases reuse.
-//  E2  one thread per (2 channels, 16-row block): alpha = exp(log_alpha), block-local
-//      running products, and from them k gamma, s q gamma (tensor-core operand) and the
-//      update operand.
+// Intra-chunk kernel, per (chunk, head), instantiated per gate form:
+//  IN  one thread loads the chunk's gate tile (log_alpha fp32, or the fused gate's f), k and q
+//      by TMA into shared memory that later phases reuse (a scalar gate is read like beta);
+//      with unit-length keys / queries asked for, the rows' norms are summed from the tiles.
+//  E2  one thread per (2 channels, 16-row block): log_alpha (computed from f for the fused
+//      gate), alpha = exp(log_alpha), block-local running products, and from them k gamma,
+//      s q gamma (tensor-core operand) and the update operand.
 //  AP  Fast path -- every channel's decay over the chunk within e^-80: A and P from one
 //      tcgen05 product [k gamma; s q gamma] (k e^-g)^T, and the update operand is
 //      k e^-g (the state update becomes Diag(gamma_last)(S + (k e^-g)^T u), its decay
@@ -1118,7 +1119,6 @@ __global__ void __launch_bounds__(SCAN_THREADS, 1)
 // threads that both find it clear both run the set-up, which is harmless.
 constexpr int kMaxDevices = 64;
 std::atomic<bool> g_configured[kMaxDevices] = {};
-std::atomic<bool> g_pool_configured[kMaxDevices] = {};
 
 using IntraKernel = void (*)(KdaChunkArgs, uint8_t *, const int32_t *, const CUtensorMap, const CUtensorMap,
                              const CUtensorMap);
@@ -1149,21 +1149,6 @@ cudaError_t configure(int dev) {
     e = cudaFuncSetAttribute(kda_chunk_scan_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kScanSmem);
     if (e != cudaSuccess) return e;
     if (dev >= 0 && dev < kMaxDevices) g_configured[dev].store(true, std::memory_order_release);
-    return cudaSuccess;
-}
-
-// Keep freed workspace in the device's default pool between calls instead of returning
-// it to the driver.
-cudaError_t configure_pool(int dev) {
-    if (dev >= 0 && dev < kMaxDevices && g_pool_configured[dev].load(std::memory_order_acquire))
-        return cudaSuccess;
-    cudaMemPool_t pool;
-    cudaError_t e = cudaDeviceGetDefaultMemPool(&pool, dev);
-    if (e != cudaSuccess) return e;
-    uint64_t keep = ~0ull;
-    e = cudaMemPoolSetAttribute(pool, cudaMemPoolAttrReleaseThreshold, &keep);
-    if (e != cudaSuccess) return e;
-    if (dev >= 0 && dev < kMaxDevices) g_pool_configured[dev].store(true, std::memory_order_release);
     return cudaSuccess;
 }
 
@@ -1280,7 +1265,7 @@ cudaError_t kda_launch_chunk_tc(const KdaChunkArgs &a, cudaStream_t stream) {
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return e;
     if ((e = configure(dev)) != cudaSuccess) return e;
-    if ((e = configure_pool(dev)) != cudaSuccess) return e;
+    if ((e = kda_keep_pool_memory(dev)) != cudaSuccess) return e;
     void *ws = nullptr;
     if ((e = cudaMallocAsync(&ws, kda_chunk_tc_workspace_bytes(a), stream)) != cudaSuccess) return e;
     e = kda_launch_chunk_tc_ws(a, ws, stream);

@@ -131,4 +131,7 @@ cudaError_t kda_launch_chunk_bwd(const KdaChunkArgs &a, int dtype, const void *d
                                  void *ws, cudaStream_t stream);
 cudaError_t kda_read_device_status(unsigned int *status, bool clear);
 cudaError_t kda_decode_read_status(unsigned int *status, bool clear);
+// Raises the release threshold of device `dev`'s default memory pool once, so that workspace
+// freed with cudaFreeAsync stays in the pool between calls (kda_api.cu).
+cudaError_t kda_keep_pool_memory(int dev);
 cudaError_t kda_launch_wait_selftest(int limit_us, cudaStream_t stream);
