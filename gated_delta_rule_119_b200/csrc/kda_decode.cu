@@ -16,10 +16,11 @@
 // calls of one token.
 //
 // Memory-bound: each state (dk x dv fp32) is read once before the first token and written
-// once after the last, whatever L is; between tokens it stays in registers.  One CTA of 256
-// threads per (n, h).  Thread (rg, cg) holds the float4 column group cg of rows rg, rg + RG,
-// ...; a warp therefore reads whole 512-byte rows, so every load and store of the state is
-// a fully coalesced 128-bit access.
+// once after the last, whatever L is; between tokens it stays in registers.  Three kernels:
+// the one-token step with the per-channel gate and no flags, one token of any other form, and
+// L tokens.  One CTA of 256 threads per (n, h).  Thread (rg, cg) holds the float4 column group
+// cg of the rows rg * ROWS .. rg * ROWS + ROWS - 1; a warp therefore reads whole 512-byte rows,
+// so every load and store of the state is a fully coalesced 128-bit access.
 #include "kda_common.cuh"
 
 // Bit 1: a sequence's state index was >= the pool size (the sequence was skipped).
@@ -29,12 +30,62 @@ namespace {
 
 constexpr int kDecodeThreads = 256;
 
-__device__ __forceinline__ float4 fma4(float s, float4 a, float4 acc) {
-    acc.x = fmaf(s, a.x, acc.x);
-    acc.y = fmaf(s, a.y, acc.y);
-    acc.z = fmaf(s, a.z, acc.z);
-    acc.w = fmaf(s, a.w, acc.w);
-    return acc;
+// The per-row arithmetic of both step kernels, on packed fp32 pairs (fma.rn.f32x2 and
+// mul.rn.f32x2 round each lane exactly as fmaf and a plain product do; one instruction does
+// two lanes).  A thread holds ROWS consecutive state rows (a warp reads ROWS whole rows), so the
+// row scalars (alpha, k, s q) come from shared memory four at a time.
+
+// Row s of the state decayed in place by al, and its share of the lookups r_k, r_q.
+__device__ __forceinline__ void decay_lookup(float4 &s, float al, float k, float q, float4 &rk, float4 &rq) {
+    const float2 a2 = make_float2(al, al), k2 = make_float2(k, k), q2 = make_float2(q, q);
+    const float2 lo = __fmul2_rn(make_float2(s.x, s.y), a2), hi = __fmul2_rn(make_float2(s.z, s.w), a2);
+    s = make_float4(lo.x, lo.y, hi.x, hi.y);
+    const float2 klo = __ffma2_rn(k2, lo, make_float2(rk.x, rk.y)), khi = __ffma2_rn(k2, hi, make_float2(rk.z, rk.w));
+    const float2 qlo = __ffma2_rn(q2, lo, make_float2(rq.x, rq.y)), qhi = __ffma2_rn(q2, hi, make_float2(rq.z, rq.w));
+    rk = make_float4(klo.x, klo.y, khi.x, khi.y);
+    rq = make_float4(qlo.x, qlo.y, qhi.x, qhi.y);
+}
+
+// The write of row s: s + k u.
+__device__ __forceinline__ float4 write_row(float4 s, float k, float4 u) {
+    const float2 k2 = make_float2(k, k);
+    const float2 lo = __ffma2_rn(k2, make_float2(u.x, u.y), make_float2(s.x, s.y));
+    const float2 hi = __ffma2_rn(k2, make_float2(u.z, u.w), make_float2(s.z, s.w));
+    return make_float4(lo.x, lo.y, hi.x, hi.y);
+}
+
+__device__ __forceinline__ float4 add4(float4 a, float4 b) {
+    const float2 lo = __fadd2_rn(make_float2(a.x, a.y), make_float2(b.x, b.y));
+    const float2 hi = __fadd2_rn(make_float2(a.z, a.w), make_float2(b.z, b.w));
+    return make_float4(lo.x, lo.y, hi.x, hi.y);
+}
+
+// V consecutive row scalars from shared memory (V = 4: one 16-byte load).
+template <int V>
+__device__ __forceinline__ void rows_of(const float *p, float *out) {
+    if constexpr (V == 4) {
+        const float4 x = *reinterpret_cast<const float4 *>(p);
+        out[0] = x.x; out[1] = x.y; out[2] = x.z; out[3] = x.w;
+    } else {
+#pragma unroll
+        for (int j = 0; j < V; ++j) out[j] = p[j];
+    }
+}
+
+// Decay the thread's rows r0 .. r0 + ROWS - 1 and form their shares of r_k and r_q.
+template <int ROWS>
+__device__ __forceinline__ void decay_lookup_rows(float4 *s, const float *sa, const float *sk, const float *sq,
+                                                  int r0, float4 &rk, float4 &rq) {
+    constexpr int V = ROWS % 4 == 0 ? 4 : 1;
+#pragma unroll
+    for (int i = 0; i < ROWS; i += V) {
+        float av[V], kv[V], qv[V];
+        rows_of<V>(sa + r0 + i, av);
+        rows_of<V>(sk + r0 + i, kv);
+        rows_of<V>(sq + r0 + i, qv);
+#pragma unroll
+        for (int j = 0; j < V; ++j) decay_lookup(s[i + j], av[j], kv[j], qv[j], rk, rq);
+    }
 }
 
 // The common step -- one token per sequence, the per-channel gate, no flags -- in its own
@@ -44,7 +95,7 @@ template <typename Tin, int DK, int DV>
 __global__ void __launch_bounds__(kDecodeThreads) kda_decode_step_kernel(KdaDecodeArgs a) {
     constexpr int CG = DV / 4, RG = kDecodeThreads / CG, ROWS = DK / RG;
     static_assert(kDecodeThreads % CG == 0 && DK % RG == 0, "decode tiling");
-    __shared__ float s_k[DK], s_q[DK], s_a[DK], s_v[DV];
+    __shared__ __align__(16) float s_k[DK], s_q[DK], s_a[DK], s_v[DV];
     __shared__ float4 s_red[2][RG][CG];
     __shared__ float s_kq;
 
@@ -61,7 +112,7 @@ __global__ void __launch_bounds__(kDecodeThreads) kda_decode_step_kernel(KdaDeco
     float4 *S4 = reinterpret_cast<float4 *>(a.S + ((size_t)idx * H + h) * DK * DV);
     float4 s[ROWS];
 #pragma unroll
-    for (int i = 0; i < ROWS; ++i) s[i] = __ldcs(&S4[(size_t)(rg + i * RG) * CG + cg]);
+    for (int i = 0; i < ROWS; ++i) s[i] = __ldcs(&S4[(size_t)(rg * ROWS + i) * CG + cg]);
 
     const Tin *qp = static_cast<const Tin *>(a.q) + (size_t)pair * DK;
     const Tin *kp = static_cast<const Tin *>(a.k) + (size_t)pair * DK;
@@ -83,17 +134,7 @@ __global__ void __launch_bounds__(kDecodeThreads) kda_decode_step_kernel(KdaDeco
         if (tid == 0) s_kq = acc;
     }
     float4 rk = make_float4(0.f, 0.f, 0.f, 0.f), rq = rk;
-#pragma unroll
-    for (int i = 0; i < ROWS; ++i) {
-        const int r = rg + i * RG;
-        const float al = s_a[r];
-        s[i].x *= al;
-        s[i].y *= al;
-        s[i].z *= al;
-        s[i].w *= al;
-        rk = fma4(s_k[r], s[i], rk);
-        rq = fma4(s_q[r], s[i], rq);
-    }
+    decay_lookup_rows<ROWS>(s, s_a, s_k, s_q, rg * ROWS, rk, rq);
     s_red[0][rg][cg] = rk;
     s_red[1][rg][cg] = rq;
     __syncthreads();
@@ -101,9 +142,8 @@ __global__ void __launch_bounds__(kDecodeThreads) kda_decode_step_kernel(KdaDeco
     float4 tk = make_float4(0.f, 0.f, 0.f, 0.f), tq = tk;
 #pragma unroll 8
     for (int g = 0; g < RG; ++g) {
-        const float4 x = s_red[0][g][cg], y = s_red[1][g][cg];
-        tk.x += x.x; tk.y += x.y; tk.z += x.z; tk.w += x.w;
-        tq.x += y.x; tq.y += y.y; tq.z += y.z; tq.w += y.w;
+        tk = add4(tk, s_red[0][g][cg]);
+        tq = add4(tq, s_red[1][g][cg]);
     }
     const float b = a.beta[pair];
     float4 u;
@@ -113,8 +153,8 @@ __global__ void __launch_bounds__(kDecodeThreads) kda_decode_step_kernel(KdaDeco
     u.w = b * (s_v[4 * cg + 3] - tk.w);
 #pragma unroll
     for (int i = 0; i < ROWS; ++i) {
-        const int r = rg + i * RG;
-        __stcs(&S4[(size_t)r * CG + cg], fma4(s_k[r], u, s[i]));
+        const int r = rg * ROWS + i;
+        __stcs(&S4[(size_t)r * CG + cg], write_row(s[i], s_k[r], u));
     }
     if (rg == 0) {
         const float kq = s_kq;
@@ -126,17 +166,22 @@ __global__ void __launch_bounds__(kDecodeThreads) kda_decode_step_kernel(KdaDeco
     }
 }
 
-// Any step: L tokens per sequence, every gate form, flags.
-template <typename Tin, int DK, int DV>
-__global__ void __launch_bounds__(kDecodeThreads) kda_decode_kernel(KdaDecodeArgs a) {
+// Any step: L tokens per sequence, every gate form, flags.  The tokens' inputs are staged in
+// shared memory LB at a time, in one pass issued right after the state loads, and the
+// per-token scalars (k . s q and the norm factors) of a batch are formed by one warp per
+// token, so the token loop itself reads no global memory.  The reduction scratch alternates
+// between two buffers from token to token: one barrier per token.
+template <typename Tin, int DK, int DV, int LB>
+__device__ __forceinline__ void decode_tokens(const KdaDecodeArgs &a) {
     constexpr int CG = DV / 4;                 // float4 column groups per state row
     constexpr int RG = kDecodeThreads / CG;    // row groups
     constexpr int ROWS = DK / RG;              // state rows per thread
     static_assert(kDecodeThreads % CG == 0 && DK % RG == 0, "decode tiling");
+    static_assert(LB <= kDecodeThreads / 32, "one warp per staged token");
 
-    __shared__ float s_k[DK], s_q[DK], s_a[DK], s_v[DV];
-    __shared__ float4 s_red[2][RG][CG];
-    __shared__ float s_fk, s_fq, s_kq;
+    __shared__ __align__(16) float s_k[LB][DK], s_q[LB][DK], s_a[LB][DK], s_v[LB][DV];
+    __shared__ float4 s_red[2][2][RG][CG];
+    __shared__ float s_fk[LB], s_fq[LB], s_kq[LB], s_b[LB];
 
     const int H = a.H;
     const int n = blockIdx.x / H, h = blockIdx.x % H;
@@ -146,14 +191,14 @@ __global__ void __launch_bounds__(kDecodeThreads) kda_decode_kernel(KdaDecodeArg
         if (threadIdx.x == 0) atomicOr(&g_kda_decode_status, 1u);
         return;
     }
-    const int tid = threadIdx.x;
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int cg = tid % CG, rg = tid / CG;
     float4 *S4 = reinterpret_cast<float4 *>(a.S + ((size_t)idx * H + h) * DK * DV);
 
     // The state is the traffic that matters: issue all of this thread's loads first.
     float4 s[ROWS];
 #pragma unroll
-    for (int i = 0; i < ROWS; ++i) s[i] = __ldcs(&S4[(size_t)(rg + i * RG) * CG + cg]);
+    for (int i = 0; i < ROWS; ++i) s[i] = __ldcs(&S4[(size_t)(rg * ROWS + i) * CG + cg]);
 
     const Tin *qg = static_cast<const Tin *>(a.q);
     const Tin *kg = static_cast<const Tin *>(a.k);
@@ -162,25 +207,33 @@ __global__ void __launch_bounds__(kDecodeThreads) kda_decode_kernel(KdaDecodeArg
     const int L = a.L, flags = a.flags, gate_kind = a.gate_kind;
     const bool norm_k = flags & kda::FLAG_NORM_K, norm_q = flags & kda::FLAG_NORM_Q;
 
-    for (int l = 0; l < L; ++l) {
-        const size_t th = ((size_t)n * L + l) * H + h;        // token-head row
-        for (int c = tid; c < DK; c += kDecodeThreads) {
-            s_k[c] = kda::to_f32(kg[th * DK + c]);
-            s_q[c] = a.scale * kda::to_f32(qg[th * DK + c]);
-            s_a[c] = expf(kda::gate_log_alpha<Tin>(gate_kind, a.gate, a.A_log, a.dt_bias, th, h, c, DK));
+    for (int l0 = 0; l0 < L; l0 += LB) {
+        const int nb = L - l0 < LB ? L - l0 : LB;
+        if (l0 > 0) __syncthreads();           // the previous batch is no longer read
+        for (int e = tid; e < nb * DK; e += kDecodeThreads) {
+            const int l = e / DK, c = e - l * DK;
+            const size_t th = ((size_t)n * L + l0 + l) * H + h;
+            s_k[l][c] = kda::to_f32(kg[th * DK + c]);
+            s_q[l][c] = a.scale * kda::to_f32(qg[th * DK + c]);
+            s_a[l][c] = expf(kda::gate_log_alpha<Tin>(gate_kind, a.gate, a.A_log, a.dt_bias, th, h, c, DK));
         }
-        for (int j = tid; j < DV; j += kDecodeThreads) s_v[j] = kda::to_f32(vg[th * DV + j]);
+        for (int e = tid; e < nb * DV; e += kDecodeThreads) {
+            const int l = e / DV, j = e - l * DV;
+            s_v[l][j] = kda::to_f32(vg[(((size_t)n * L + l0 + l) * H + h) * DV + j]);
+        }
+        if (tid < nb) s_b[tid] = kda::beta_of(a.beta[((size_t)n * L + l0 + tid) * H + h], flags);
         __syncthreads();
 
-        if (tid < 32) {                        // k . q and, when asked for, the norms: one warp
+        if (warp < nb) {                       // k . q and, when asked for, the norms: one warp a token
+            const int l = warp;
             float kq = 0.f, kk = 0.f, qq = 0.f;
-            for (int c = tid; c < DK; c += 32) kq = fmaf(s_k[c], s_q[c], kq);
+            for (int c = lane; c < DK; c += 32) kq = fmaf(s_k[l][c], s_q[l][c], kq);
 #pragma unroll
             for (int o = 16; o > 0; o >>= 1) kq += __shfl_xor_sync(0xffffffffu, kq, o);
             if (norm_k || norm_q) {
-                for (int c = tid; c < DK; c += 32) {
-                    kk = fmaf(s_k[c], s_k[c], kk);
-                    qq = fmaf(s_q[c], s_q[c], qq);
+                for (int c = lane; c < DK; c += 32) {
+                    kk = fmaf(s_k[l][c], s_k[l][c], kk);
+                    qq = fmaf(s_q[l][c], s_q[l][c], qq);
                 }
 #pragma unroll
                 for (int o = 16; o > 0; o >>= 1) {
@@ -188,61 +241,67 @@ __global__ void __launch_bounds__(kDecodeThreads) kda_decode_kernel(KdaDecodeArg
                     qq += __shfl_xor_sync(0xffffffffu, qq, o);
                 }
             }
-            if (tid == 0) {
+            if (lane == 0) {
                 // s_q holds s q, so 1 / max(||q||, eps) = s / max(||s q||, s eps)
                 const float fk = norm_k ? 1.f / fmaxf(sqrtf(kk), 1e-12f) : 1.f;
                 const float fq = norm_q ? a.scale / fmaxf(sqrtf(qq), a.scale * 1e-12f) : 1.f;
-                s_fk = fk;
-                s_fq = fq;
-                s_kq = fk * fq * kq;
+                s_fk[l] = fk;
+                s_fq[l] = fq;
+                s_kq[l] = fk * fq * kq;
             }
         }
 
-        float4 rk = make_float4(0.f, 0.f, 0.f, 0.f), rq = rk;
-#pragma unroll
-        for (int i = 0; i < ROWS; ++i) {
-            const int r = rg + i * RG;
-            const float al = s_a[r];
-            s[i].x *= al;
-            s[i].y *= al;
-            s[i].z *= al;
-            s[i].w *= al;
-            rk = fma4(s_k[r], s[i], rk);
-            rq = fma4(s_q[r], s[i], rq);
-        }
-        s_red[0][rg][cg] = rk;
-        s_red[1][rg][cg] = rq;
-        __syncthreads();
+        for (int l = 0; l < nb; ++l) {
+            const size_t th = ((size_t)n * L + l0 + l) * H + h;   // token-head row
+            const int par = l & 1;
+            float4 rk = make_float4(0.f, 0.f, 0.f, 0.f), rq = rk;
+            decay_lookup_rows<ROWS>(s, s_a[l], s_k[l], s_q[l], rg * ROWS, rk, rq);
+            s_red[par][0][rg][cg] = rk;
+            s_red[par][1][rg][cg] = rq;
+            __syncthreads();                   // also publishes the batch's per-token scalars
 
-        float4 tk = make_float4(0.f, 0.f, 0.f, 0.f), tq = tk;
+            float4 tk = make_float4(0.f, 0.f, 0.f, 0.f), tq = tk;
 #pragma unroll 8
-        for (int g = 0; g < RG; ++g) {
-            const float4 x = s_red[0][g][cg], y = s_red[1][g][cg];
-            tk.x += x.x; tk.y += x.y; tk.z += x.z; tk.w += x.w;
-            tq.x += y.x; tq.y += y.y; tq.z += y.z; tq.w += y.w;
-        }
-        const float fk = s_fk, fq = s_fq;
-        const float b = kda::beta_of(a.beta[th], flags);
-        float4 u;
-        u.x = b * (s_v[4 * cg + 0] - fk * tk.x);
-        u.y = b * (s_v[4 * cg + 1] - fk * tk.y);
-        u.z = b * (s_v[4 * cg + 2] - fk * tk.z);
-        u.w = b * (s_v[4 * cg + 3] - fk * tk.w);
-        const float4 uk = make_float4(fk * u.x, fk * u.y, fk * u.z, fk * u.w);
+            for (int g = 0; g < RG; ++g) {
+                tk = add4(tk, s_red[par][0][g][cg]);
+                tq = add4(tq, s_red[par][1][g][cg]);
+            }
+            const float fk = s_fk[l], fq = s_fq[l];
+            const float b = s_b[l];
+            const float *vv = s_v[l];
+            float4 u;
+            u.x = b * (vv[4 * cg + 0] - fk * tk.x);
+            u.y = b * (vv[4 * cg + 1] - fk * tk.y);
+            u.z = b * (vv[4 * cg + 2] - fk * tk.z);
+            u.w = b * (vv[4 * cg + 3] - fk * tk.w);
+            const float4 uk = make_float4(fk * u.x, fk * u.y, fk * u.z, fk * u.w);
 #pragma unroll
-        for (int i = 0; i < ROWS; ++i) s[i] = fma4(s_k[rg + i * RG], uk, s[i]);
-        if (rg == 0) {
-            const float kq = s_kq;
-            Tin *op = og + th * DV + 4 * cg;
-            op[0] = kda::from_f32<Tin>(fmaf(u.x, kq, fq * tq.x));
-            op[1] = kda::from_f32<Tin>(fmaf(u.y, kq, fq * tq.y));
-            op[2] = kda::from_f32<Tin>(fmaf(u.z, kq, fq * tq.z));
-            op[3] = kda::from_f32<Tin>(fmaf(u.w, kq, fq * tq.w));
+            for (int i = 0; i < ROWS; ++i) s[i] = write_row(s[i], s_k[l][rg * ROWS + i], uk);
+            if (rg == 0) {
+                const float kq = s_kq[l];
+                Tin *op = og + th * DV + 4 * cg;
+                op[0] = kda::from_f32<Tin>(fmaf(u.x, kq, fq * tq.x));
+                op[1] = kda::from_f32<Tin>(fmaf(u.y, kq, fq * tq.y));
+                op[2] = kda::from_f32<Tin>(fmaf(u.z, kq, fq * tq.z));
+                op[3] = kda::from_f32<Tin>(fmaf(u.w, kq, fq * tq.w));
+            }
         }
-        if (l + 1 < L) __syncthreads();         // the next token's inputs reuse shared memory
     }
 #pragma unroll
-    for (int i = 0; i < ROWS; ++i) __stcs(&S4[(size_t)(rg + i * RG) * CG + cg], s[i]);
+    for (int i = 0; i < ROWS; ++i) __stcs(&S4[(size_t)(rg * ROWS + i) * CG + cg], s[i]);
+}
+
+// L tokens, staged four at a time.
+template <typename Tin, int DK, int DV>
+__global__ void __launch_bounds__(kDecodeThreads) kda_decode_kernel(KdaDecodeArgs a) {
+    decode_tokens<Tin, DK, DV, 4>(a);
+}
+
+// One token with a gate form or flags the step kernel does not take: three CTAs per SM (a few
+// registers spill), so one CTA's state loads overlap another's arithmetic.
+template <typename Tin, int DK, int DV>
+__global__ void __launch_bounds__(kDecodeThreads, 3) kda_decode_single_kernel(KdaDecodeArgs a) {
+    decode_tokens<Tin, DK, DV, 1>(a);
 }
 
 template <typename Tin, int DK, int DV>
@@ -250,6 +309,8 @@ cudaError_t launch(const KdaDecodeArgs &a, cudaStream_t st) {
     const unsigned grid = (unsigned)((int64_t)a.N * a.H);
     if (a.L == 1 && a.gate_kind == kda::GATE_CHANNEL && a.flags == 0)
         kda_decode_step_kernel<Tin, DK, DV><<<grid, kDecodeThreads, 0, st>>>(a);
+    else if (a.L == 1)
+        kda_decode_single_kernel<Tin, DK, DV><<<grid, kDecodeThreads, 0, st>>>(a);
     else
         kda_decode_kernel<Tin, DK, DV><<<grid, kDecodeThreads, 0, st>>>(a);
     return cudaGetLastError();

@@ -214,9 +214,11 @@ def test_decode_padding_leaves_out_untouched():
 
 @pytest.mark.parametrize("dtype", ["f32", "bf16"])
 @pytest.mark.parametrize("form,raw", [("channel", False), ("fused", True)])
-def test_multi_token_step_equals_single_steps(dtype, form, raw):
-    """One call over L = 4 tokens == four calls of one token each, bit for bit."""
-    N, L, H, d, P = 5, 4, 2, 128, 9
+@pytest.mark.parametrize("L", [4, 7])
+def test_multi_token_step_equals_single_steps(dtype, form, raw, L):
+    """One call over L tokens == L calls of one token each, bit for bit (L = 7 spans two
+    batches of staged tokens, the second one partial)."""
+    N, H, d, P = 5, 2, 128, 9
     inp = _decode_case(N, L, H, d, dtype, 520, form, raw)
     t = to_torch(inp)
     idx = torch.tensor([4, 0, 8, 2, 6], dtype=torch.int32, device="cuda")
