@@ -37,7 +37,9 @@ constexpr int kC = 16;
 static_assert(kThreads == 32 * kC, "the K / P and gradient passes map warp w to row or column w, lane to a channel group");
 
 // Row pitches are padded to a multiple of 4 floats so that rows can be read 16 bytes at a time.
-template <int DK, int DVH>
+// ES is the input element size; the staging area at the end holds the next chunk's raw inputs
+// (k, q, the gate, v, dO, beta), copied in while the current chunk is computed.
+template <int DK, int DVH, int ES>
 struct BwdLayout {
     static constexpr int LK = DK + 4, LV = DVH + 4, LC = kC + 1;
     // [kC][LK] arrays
@@ -54,7 +56,13 @@ struct BwdLayout {
                          DTM = DPM + kC * LC, XM = DTM + kC * LC;
     static constexpr int GC = XM + kC * LC, BT = GC + DK, DB = BT + kC, DGC = DB + kC;
     static constexpr int DGP = DGC + DK;      // [kThreads / DK][DK] partial last-row g terms
-    static constexpr int floats = DGP + kThreads;
+    // staging, in bytes from its start: k, q [kC][DK] and v, dO [kC][DVH] in the input type, the
+    // gate [kC][DK] fp32 (a scalar gate uses [kC]), beta [kC]
+    static constexpr int ST = DGP + kThreads;
+    static constexpr int ST_K = 0, ST_Q = ST_K + kC * DK * ES, ST_G = ST_Q + kC * DK * ES,
+                         ST_V = ST_G + kC * DK * 4, ST_DO = ST_V + kC * DVH * ES, ST_B = ST_DO + kC * DVH * ES,
+                         ST_BYTES = ST_B + kC * 4;
+    static constexpr int floats = ST + ST_BYTES / 4;
     static constexpr size_t bytes = (size_t)floats * sizeof(float);
 };
 
@@ -77,6 +85,18 @@ __device__ __forceinline__ size_t part_index(const BwdArgs &b, int split, size_t
 
 __device__ __forceinline__ float4 ld4(const float *p) { return *reinterpret_cast<const float4 *>(p); }
 
+// Asynchronous global -> shared copies (16 bytes, or 4 for the strided per-token scalars).
+__device__ __forceinline__ void cp_async16(void *dst, const void *src) {
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"((uint32_t)__cvta_generic_to_shared(dst)),
+                 "l"(src) : "memory");
+}
+__device__ __forceinline__ void cp_async4(void *dst, const void *src) {
+    asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"((uint32_t)__cvta_generic_to_shared(dst)),
+                 "l"(src) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+__device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_all;" ::: "memory"); }
+
 // acc += a . b over four consecutive k, in k order.
 __device__ __forceinline__ float dot4(float4 a, float4 b, float acc) {
     return fmaf(a.w, b.w, fmaf(a.z, b.z, fmaf(a.y, b.y, fmaf(a.x, b.x, acc))));
@@ -84,7 +104,7 @@ __device__ __forceinline__ float dot4(float4 a, float4 b, float acc) {
 
 template <typename Tin, int DK, int DVH>
 __global__ void __launch_bounds__(kThreads, 1) kda_chunk_bwd_kernel(BwdArgs b) {   // 16 warps, <= 128 registers
-    using L = BwdLayout<DK, DVH>;
+    using L = BwdLayout<DK, DVH, (int)sizeof(Tin)>;
     constexpr int LK = L::LK, LV = L::LV, LC = L::LC, CH = kC;
     constexpr int RPT = kC * DVH / kThreads;   // rows per thread of the [C][dv] products
     constexpr int CPT = DK * DVH / kThreads;   // rows per thread of the [dk][dv] products
@@ -99,6 +119,7 @@ __global__ void __launch_bounds__(kThreads, 1) kda_chunk_bwd_kernel(BwdArgs b) {
     float *KM = sm + L::KM, *TM = sm + L::TM, *PM = sm + L::PM, *DPM = sm + L::DPM, *DTM = sm + L::DTM;
     float *XM = sm + L::XM, *GC = sm + L::GC, *BT = sm + L::BT, *DB = sm + L::DB, *DGC = sm + L::DGC;
     float *DGP = sm + L::DGP;
+    uint8_t *STG = reinterpret_cast<uint8_t *>(sm + L::ST);
 
     const KdaChunkArgs &a = b.a;
     const int H = a.H, dv = a.dv;
@@ -137,38 +158,87 @@ __global__ void __launch_bounds__(kThreads, 1) kda_chunk_bwd_kernel(BwdArgs b) {
     };
     const size_t sbase = (size_t)pair * DK * dv;
 
-    for (int idx = tid; idx < DK * DVH; idx += kThreads) {
-        const int c = idx / DVH, j = idx % DVH;
-        S[c * LV + j] = a.S0 ? a.S0[sbase + (size_t)c * dv + j0 + j] : 0.f;
-        DS[c * LV + j] = b.dS_final ? b.dS_final[sbase + (size_t)c * dv + j0 + j] : 0.f;
+#pragma unroll 4
+    for (int v4 = tid; v4 < DK * DVH / 4; v4 += kThreads) {
+        const int c = 4 * v4 / DVH, j = 4 * v4 % DVH;
+        const float4 z = make_float4(0.f, 0.f, 0.f, 0.f);
+        *reinterpret_cast<float4 *>(S + c * LV + j) = a.S0 ? ld4(a.S0 + sbase + (size_t)c * dv + j0 + j) : z;
+        *reinterpret_cast<float4 *>(DS + c * LV + j) = b.dS_final ? ld4(b.dS_final + sbase + (size_t)c * dv + j0 + j) : z;
     }
+
+    // Issues the copies of chunk c0's raw inputs into the staging area (rows < nr; q and dO
+    // only for the backward pass).  Consumed by chunk_terms after a wait.
+    auto prefetch = [&](int64_t c0, int nr, bool with_q) {
+        constexpr int KCH = DK * (int)sizeof(Tin) / 16, GCH = DK * 4 / 16, VCH = DVH * (int)sizeof(Tin) / 16;
+        for (int idx = tid; idx < nr * KCH; idx += kThreads) {
+            const int r = idx / KCH, q16 = idx % KCH;
+            const size_t off = ((size_t)(c0 + r) * H + h) * DK * sizeof(Tin) + 16 * q16;
+            cp_async16(STG + L::ST_K + r * DK * (int)sizeof(Tin) + 16 * q16, reinterpret_cast<const uint8_t *>(kg) + off);
+            if (with_q)
+                cp_async16(STG + L::ST_Q + r * DK * (int)sizeof(Tin) + 16 * q16,
+                           reinterpret_cast<const uint8_t *>(qg) + off);
+        }
+        if (a.gate_kind == kda::GATE_CHANNEL) {
+            for (int idx = tid; idx < nr * GCH; idx += kThreads) {
+                const int r = idx / GCH, q16 = idx % GCH;
+                cp_async16(STG + L::ST_G + r * DK * 4 + 16 * q16,
+                           static_cast<const uint8_t *>(a.gate) + ((size_t)(c0 + r) * H + h) * DK * 4 + 16 * q16);
+            }
+        } else if (a.gate_kind == kda::GATE_SCALAR && tid < nr) {
+            cp_async4(STG + L::ST_G + 4 * tid, static_cast<const float *>(a.gate) + (size_t)(c0 + tid) * H + h);
+        }
+        for (int idx = tid; idx < nr * VCH; idx += kThreads) {
+            const int r = idx / VCH, q16 = idx % VCH;
+            const size_t off = (((size_t)(c0 + r) * H + h) * dv + j0) * sizeof(Tin) + 16 * q16;
+            cp_async16(STG + L::ST_V + r * DVH * (int)sizeof(Tin) + 16 * q16, reinterpret_cast<const uint8_t *>(vg) + off);
+            if (with_q)
+                cp_async16(STG + L::ST_DO + r * DVH * (int)sizeof(Tin) + 16 * q16,
+                           reinterpret_cast<const uint8_t *>(dog) + off);
+        }
+        if (tid < nr) cp_async4(STG + L::ST_B + 4 * tid, a.beta + (size_t)(c0 + tid) * H + h);
+        cp_async_commit();
+    };
     __syncthreads();
 
-    // Loads chunk c0's rows (zeros / alpha = 1 / beta = 0 past the sequence end) and forms the
-    // decay products and the chunk matrices K, T (and P with `with_p`).
-    auto chunk_terms = [&](int64_t c0, int nr, bool with_q) {
-        for (int idx = tid; idx < CH * DK; idx += kThreads) {
-            const int r = idx / DK, c = idx % DK;
-            float kv = 0.f, qv = 0.f, al = 1.f;
-            if (r < nr) {
-                const size_t th = (size_t)(c0 + r) * H + h, off = th * DK + c;
-                kv = kda::to_f32(kg[off]);
-                qv = with_q ? kda::to_f32(qg[off]) : 0.f;
-                al = expf(kda::gate_log_alpha<Tin>(a.gate_kind, a.gate, a.A_log, a.dt_bias, th, h, c, DK));
+    // Takes chunk c0's rows from the staging area (zeros / alpha = 1 / beta = 0 past the sequence
+    // end; with_q: also q and dO), starts the copies of the next chunk (pf_nr rows from pf_c0,
+    // none when pf_nr = 0), and forms the decay products and the chunk matrices K, T, P.
+    auto chunk_terms = [&](int64_t c0, int nr, bool with_q, int64_t pf_c0, int pf_nr, bool pf_q) {
+        cp_async_wait_all();
+        __syncthreads();                       // this chunk's staged rows are visible to all
+        {
+            const Tin *sk = reinterpret_cast<const Tin *>(STG + L::ST_K), *sq = reinterpret_cast<const Tin *>(STG + L::ST_Q);
+            const Tin *sv = reinterpret_cast<const Tin *>(STG + L::ST_V), *sdo = reinterpret_cast<const Tin *>(STG + L::ST_DO);
+            const float *sg = reinterpret_cast<const float *>(STG + L::ST_G), *sb = reinterpret_cast<const float *>(STG + L::ST_B);
+#pragma unroll
+            for (int it = 0; it < CH * DK / kThreads; ++it) {
+                const int idx = tid + it * kThreads, r = idx / DK, c = idx % DK;
+                float kv = 0.f, qv = 0.f, al = 1.f;
+                if (r < nr) {
+                    kv = kda::to_f32(sk[r * DK + c]);
+                    qv = with_q ? kda::to_f32(sq[r * DK + c]) : 0.f;
+                    const float la = a.gate_kind == kda::GATE_CHANNEL ? sg[r * DK + c]
+                                     : (a.gate_kind == kda::GATE_SCALAR ? sg[r] : 0.f);
+                    al = expf(la);
+                }
+                Kk[r * LK + c] = kv;
+                Q[r * LK + c] = qv;
+                AL[r * LK + c] = al;
             }
-            Kk[r * LK + c] = kv;
-            Q[r * LK + c] = qv;
-            AL[r * LK + c] = al;
+#pragma unroll
+            for (int it = 0; it < CH * DVH / kThreads; ++it) {
+                const int idx = tid + it * kThreads, r = idx / DVH, j = idx % DVH;
+                V[r * LV + j] = r < nr ? kda::to_f32(sv[r * DVH + j]) : 0.f;
+                if (with_q) DO[r * LV + j] = r < nr ? kda::to_f32(sdo[r * DVH + j]) : 0.f;
+            }
+            if (tid < CH) BT[tid] = tid < nr ? sb[tid] : 0.f;
         }
-        for (int idx = tid; idx < CH * DVH; idx += kThreads) {
-            const int r = idx / DVH, j = idx % DVH;
-            V[r * LV + j] = r < nr ? kda::to_f32(vg[((size_t)(c0 + r) * H + h) * dv + j0 + j]) : 0.f;
-        }
-        if (tid < CH) BT[tid] = tid < nr ? a.beta[(size_t)(c0 + tid) * H + h] : 0.f;
-        __syncthreads();
+        __syncthreads();                       // the staging area is free
+        if (pf_nr > 0) prefetch(pf_c0, pf_nr, pf_q);
         // gamma (forward running product) and kappa (reverse), per channel
         for (int c = tid; c < DK; c += kThreads) {
             float g = 1.f;
+#pragma unroll
             for (int r = 0; r < CH; ++r) {
                 g *= AL[r * LK + c];
                 GA[r * LK + c] = g;
@@ -177,6 +247,7 @@ __global__ void __launch_bounds__(kThreads, 1) kda_chunk_bwd_kernel(BwdArgs b) {
             }
             GC[c] = g;
             float kp = 1.f;
+#pragma unroll
             for (int r = CH - 1; r >= 0; --r) {
                 KA[r * LK + c] = kp;
                 KK[r * LK + c] = Kk[r * LK + c] * kp;
@@ -184,49 +255,59 @@ __global__ void __launch_bounds__(kThreads, 1) kda_chunk_bwd_kernel(BwdArgs b) {
             }
         }
         // K and P: warp i, lane = channel group cg of 32, carries running products down the rows
-        // r >= i; the 32 groups of a column are summed by full-warp shuffles (every lane of the
-        // warp walks the same rows).
+        // r >= i; the 32 groups of a column are then summed by full-warp shuffles, all rows'
+        // sums together (every lane of the warp takes part).
         {
             const int i = tid >> 5, cg = tid & 31;
             constexpr int CPT = DK / 32;
-            float f[CPT];
+            float f[CPT], sk[CH], sp[CH];
 #pragma unroll
             for (int m = 0; m < CPT; ++m) f[m] = 1.f;
+#pragma unroll
             for (int r = 0; r < CH; ++r) {
-                float sk = 0.f, sp = 0.f;
+                sk[r] = 0.f;
+                sp[r] = 0.f;
                 if (r >= i) {
 #pragma unroll
                     for (int m = 0; m < CPT; ++m) {
                         const int c = cg + 32 * m;
                         if (r > i) f[m] *= AL[r * LK + c];
                         const float kd = Kk[i * LK + c] * f[m];
-                        sk = fmaf(Kk[r * LK + c], kd, sk);
-                        sp = fmaf(Q[r * LK + c], kd, sp);
+                        sk[r] = fmaf(Kk[r * LK + c], kd, sk[r]);
+                        sp[r] = fmaf(Q[r * LK + c], kd, sp[r]);
                     }
                 }
+            }
 #pragma unroll
-                for (int o = 16; o > 0; o >>= 1) {
-                    sk += __shfl_xor_sync(0xffffffffu, sk, o);
-                    sp += __shfl_xor_sync(0xffffffffu, sp, o);
+            for (int o = 16; o > 0; o >>= 1) {
+#pragma unroll
+                for (int r = 0; r < CH; ++r) {
+                    sk[r] += __shfl_xor_sync(0xffffffffu, sk[r], o);
+                    sp[r] += __shfl_xor_sync(0xffffffffu, sp[r], o);
                 }
-                if (cg == 0) {
-                    KM[r * LC + i] = r > i ? sk : 0.f;
-                    PM[r * LC + i] = r >= i ? scale * sp : 0.f;
+            }
+            if (cg == 0) {
+#pragma unroll
+                for (int r = 0; r < CH; ++r) {
+                    KM[r * LC + i] = r > i ? sk[r] : 0.f;
+                    PM[r * LC + i] = r >= i ? scale * sp[r] : 0.f;
                 }
             }
         }
         __syncthreads();
-        // T = (I + Diag(beta) K)^{-1}, unit lower triangular: column i by forward substitution
+        // T = (I + Diag(beta) K)^{-1}, unit lower triangular: column i by forward substitution,
+        // the column in registers (its entries above row i are zero, so the sums over m < i add
+        // exact zeros before the first term, as if they started at m = i)
         if (tid < CH) {
             const int i = tid;
+            float t[CH];
+#pragma unroll
             for (int r = 0; r < CH; ++r) {
-                float t = r == i ? 1.f : 0.f;
-                if (r > i) {
-                    float acc = 0.f;
-                    for (int m = i; m < r; ++m) acc = fmaf(BT[r] * KM[r * LC + m], TM[m * LC + i], acc);
-                    t = -acc;
-                }
-                TM[r * LC + i] = t;
+                float acc = 0.f;
+#pragma unroll
+                for (int m = 0; m < r; ++m) acc = fmaf(BT[r] * KM[r * LC + m], t[m], acc);
+                t[r] = r < i ? 0.f : (r == i ? 1.f : -acc);
+                TM[r * LC + i] = t[r];
             }
         }
         __syncthreads();
@@ -260,12 +341,18 @@ __global__ void __launch_bounds__(kThreads, 1) kda_chunk_bwd_kernel(BwdArgs b) {
     };
 
     // ---------------------------------------------------------------- forward: checkpoints
+    auto chunk_rows = [&](int ci) { const int64_t c0 = t0 + (int64_t)ci * CH; return (int)(t1 - c0 < CH ? t1 - c0 : CH); };
+    if (nch > 0) prefetch(t0, chunk_rows(0), false);
     for (int ci = 0; ci < nch; ++ci) {
         const int64_t c0 = t0 + (int64_t)ci * CH;
-        const int nr = (int)(t1 - c0 < CH ? t1 - c0 : CH);
+        const int nr = chunk_rows(ci);
         float *dst = ckpt_block(ci);
-        for (int idx = tid; idx < DK * DVH; idx += kThreads) dst[idx] = S[(idx / DVH) * LV + idx % DVH];
-        chunk_terms(c0, nr, false);
+#pragma unroll 4
+        for (int v4 = tid; v4 < DK * DVH / 4; v4 += kThreads)
+            *reinterpret_cast<float4 *>(dst + 4 * v4) = ld4(S + (4 * v4 / DVH) * LV + 4 * v4 % DVH);
+        // next: chunk ci + 1, or after the last one the backward pass's first chunk (the last)
+        const int nx = ci + 1 < nch ? ci + 1 : nch - 1;
+        chunk_terms(c0, nr, false, t0 + (int64_t)nx * CH, chunk_rows(nx), ci + 1 >= nch);
         // S <- Diag(gamma_last) S + (k kappa)^T u, in place.  Thread: column j, CPT rows.
         {
             const int j = tid % DVH, c0 = (tid / DVH) * CPT;
@@ -299,13 +386,10 @@ __global__ void __launch_bounds__(kThreads, 1) kda_chunk_bwd_kernel(BwdArgs b) {
         const int64_t c0 = t0 + (int64_t)ci * CH;
         const int nr = (int)(t1 - c0 < CH ? t1 - c0 : CH);
         const float *src = ckpt_block(ci);
-        for (int idx = tid; idx < DK * DVH; idx += kThreads) S[(idx / DVH) * LV + idx % DVH] = src[idx];
-        for (int idx = tid; idx < CH * DVH; idx += kThreads) {
-            const int r = idx / DVH, j = idx % DVH;
-            DO[r * LV + j] = r < nr ? kda::to_f32(dog[((size_t)(c0 + r) * H + h) * dv + j0 + j]) : 0.f;
-        }
-        __syncthreads();
-        chunk_terms(c0, nr, true);
+#pragma unroll 4
+        for (int v4 = tid; v4 < DK * DVH / 4; v4 += kThreads)
+            *reinterpret_cast<float4 *>(S + (4 * v4 / DVH) * LV + 4 * v4 % DVH) = ld4(src + 4 * v4);
+        chunk_terms(c0, nr, true, c0 - CH, ci > 0 ? CH : 0, true);
 
         // du = P^T dO + (k kappa) dS', then dr = Diag(beta) T^T du (this half's dv rows).
         // Thread: column j, RPT rows.
@@ -502,9 +586,10 @@ __global__ void __launch_bounds__(kThreads, 1) kda_chunk_bwd_kernel(BwdArgs b) {
         __syncthreads();
     }
     if (b.dS0)
-        for (int idx = tid; idx < DK * DVH; idx += kThreads) {
-            const int c = idx / DVH, j = idx % DVH;
-            b.dS0[sbase + (size_t)c * dv + j0 + j] = DS[c * LV + j];
+#pragma unroll 4
+        for (int v4 = tid; v4 < DK * DVH / 4; v4 += kThreads) {
+            const int c = 4 * v4 / DVH, j = 4 * v4 % DVH;
+            *reinterpret_cast<float4 *>(b.dS0 + sbase + (size_t)c * dv + j0 + j) = ld4(DS + c * LV + j);
         }
 }
 
@@ -545,7 +630,7 @@ __global__ void kda_chunk_bwd_reduce_kernel(BwdArgs b, void *dq_out, void *dk_ou
 
 template <typename Tin, int DK, int DVH>
 cudaError_t launch_bwd(const BwdArgs &b, cudaStream_t st) {
-    const size_t smem = BwdLayout<DK, DVH>::bytes;
+    const size_t smem = BwdLayout<DK, DVH, (int)sizeof(Tin)>::bytes;
     cudaError_t e = cudaFuncSetAttribute(kda_chunk_bwd_kernel<Tin, DK, DVH>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
