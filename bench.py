@@ -791,8 +791,11 @@ def decode_pairs(dev_in, S0, device, kda_decode_step):
 
 
 def run_e2e(args, name, device, stream, rank):
-    """The same metric through the public call with pinned host buffers: H2D of
-    the step's inputs, the call, D2H of its results, all inside the timed region."""
+    """The same metric through the public call with pinned host buffers: every step copies its
+    inputs host -> device, makes the call and copies its results back, all inside the timed
+    region.  The N sequences go in up to four groups on three streams (copies in, the calls,
+    copies out), so a group's results travel back while the next group's inputs travel in and
+    another group is computed: the host link carries both directions at once."""
     import torch
     from gated_delta_rule_119_b200 import kda_chunk_fwd, kda_decode_step
     w = WORKLOADS[name]
@@ -804,7 +807,8 @@ def run_e2e(args, name, device, stream, rank):
         S_host = torch.from_numpy(make_decode_state(N, H, dk, dv, 5)).pin_memory()
         out_host = torch.empty((N, H, dv), dtype=host["q"].dtype).pin_memory()
         S_dev = torch.empty_like(S_host, device=device)
-        units = N
+        S_dev.copy_(S_host)
+        units, cu = N, None
     else:
         inp = make_workload(name) if rank == 0 else make_inputs(
             w["B"], w["T"], w["H"], w["dk"], w["dv"], w["dtype"], rank_seed(w["index"], rank),
@@ -812,40 +816,76 @@ def run_e2e(args, name, device, stream, rank):
         host = to_torch(inp, "cpu", pin=True)
         out_host = torch.empty(host["v"].shape, dtype=host["q"].dtype).pin_memory()
         S_host = torch.empty((inp.n_seqs, inp.H, inp.dk, inp.dv), dtype=torch.float32).pin_memory()
-        units = inp.total_tokens
-    h2d = sum(t.numel() * t.element_size() for t in host.values() if t is not None)
+        N, units = inp.n_seqs, inp.total_tokens
+        cu = None if host["cu_seqlens"] is None else host["cu_seqlens"].numpy().astype(np.int64)
     # Decode keeps the recurrent state resident in HBM across steps (it is the model's
     # memory, not a step input): a step moves the new token's q, k, v and gates in and
     # its o out.  Prefill moves every input in and o plus the final states out.
-    d2h = out_host.numel() * out_host.element_size() + (0 if name == "decode" else S_host.numel() * 4)
-    if name == "decode":
-        S_dev.copy_(S_host)
+    P = min(N, 4)
+    bounds = [(N * g // P, N * (g + 1) // P) for g in range(P)]
+    groups = []
+    for b0, b1 in bounds:
+        # token tensors lead with the sequence axis, or (packed) with the group's token range
+        sl = slice(b0, b1) if cu is None else slice(int(cu[b0]), int(cu[b1]))
+        hin = {k: (None if host.get(k) is None else host[k][sl]) for k in ("q", "k", "v", "log_alpha", "beta")}
+        hin["S0"] = None if host.get("S0") is None else host["S0"][b0:b1]
+        hin["cu_seqlens"] = None if cu is None else \
+            torch.from_numpy((cu[b0:b1 + 1] - cu[b0]).astype(np.int32)).pin_memory()
+        g = {"in": hin, "dev": {k: (None if t is None else torch.empty_like(t, device=device))
+                                for k, t in hin.items()},
+             "out_h": out_host[sl], "out_d": torch.empty_like(out_host[sl], device=device)}
+        if name != "decode":
+            g["S_h"] = S_host[b0:b1]
+            g["S_d"] = torch.empty_like(g["S_h"], device=device)
+        groups.append(g)
+    h2d = sum(t.numel() * t.element_size() for g in groups for t in g["in"].values() if t is not None)
+    d2h = sum(g["out_h"].numel() * g["out_h"].element_size() + (g["S_h"].numel() * 4 if "S_h" in g else 0)
+              for g in groups)
+    s_in, s_c, s_out = (torch.cuda.Stream(device) for _ in range(3))
+    ev_i = [torch.cuda.Event() for _ in groups]   # group g's inputs are on the device
+    ev_c = [torch.cuda.Event() for _ in groups]   # group g's call is done (its input buffers are free)
+    ev_o = [torch.cuda.Event() for _ in groups]   # group g's results are home (its output buffers are free)
 
     def one():
-        d = {k: (None if t is None else t.to(device, non_blocking=True)) for k, t in host.items()}
-        if name == "decode":
-            o = kda_decode_step(d["q"], d["k"], d["v"], d["log_alpha"], d["beta"], S_dev)
-            out_host.copy_(o, non_blocking=True)
-        else:
-            o, Sf = kda_chunk_fwd(d["q"], d["k"], d["v"], d["log_alpha"], d["beta"], d["S0"],
-                                  d["cu_seqlens"])
-            out_host.copy_(o, non_blocking=True)
-            S_host.copy_(Sf, non_blocking=True)
+        for gi, (g, (b0, b1)) in enumerate(zip(groups, bounds)):
+            s_in.wait_event(ev_c[gi])
+            with torch.cuda.stream(s_in):
+                for k, t in g["in"].items():
+                    if t is not None:
+                        g["dev"][k].copy_(t, non_blocking=True)
+            ev_i[gi].record(s_in)
+            s_c.wait_event(ev_i[gi])
+            s_c.wait_event(ev_o[gi])
+            d = g["dev"]
+            if name == "decode":
+                kda_decode_step(d["q"], d["k"], d["v"], d["log_alpha"], d["beta"], S_dev[b0:b1], g["out_d"],
+                                stream=s_c)
+            else:
+                kda_chunk_fwd(d["q"], d["k"], d["v"], d["log_alpha"], d["beta"], d["S0"], d["cu_seqlens"],
+                              g["out_d"], g["S_d"], stream=s_c)
+            ev_c[gi].record(s_c)
+            s_out.wait_event(ev_c[gi])
+            with torch.cuda.stream(s_out):
+                g["out_h"].copy_(g["out_d"], non_blocking=True)
+                if "S_h" in g:
+                    g["S_h"].copy_(g["S_d"], non_blocking=True)
+            ev_o[gi].record(s_out)
 
     one()
     torch.cuda.synchronize(device)
     barrier(device)
     ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    ev0.record(stream)
+    ev0.record(s_in)
     for _ in range(steps):
         one()
-    ev1.record(stream)
+    ev1.record(s_out)                             # after the last group's results are home
     torch.cuda.synchronize(device)
     ms = reduce_max(ev0.elapsed_time(ev1) / steps, device)
     world = int(os.environ.get("WORLD_SIZE", 1))
     return {"value": units * world / (ms / 1e3), "unit": "tokens/s", "ms_per_step": ms,
             "steps": steps, "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
-            "path": "pinned host -> kda_* public call -> pinned host"
+            "path": f"pinned host -> kda_* public call -> pinned host, the sequences in {P} groups on "
+                    "three streams (copies in, calls, copies out overlapping)"
                     + (" (decode state resident in HBM)" if name == "decode" else "")}
 
 
