@@ -34,6 +34,10 @@ namespace {
 
 constexpr int kThreads = 512;
 constexpr int kC = 16;
+// A chunk whose decay stays within e^-80 in every channel (gamma_last >= e^-80) forms its decay
+// factors D[r][i][c] = gamma_r / gamma_i as products of gamma_r and 1 / gamma_i, both in
+// [1, e^80] or [e^-80, 1]: K, P and their gradients through D become plain small products.
+constexpr float kFastGammaMin = 1.8048513e-35f;   // e^-80
 static_assert(kThreads == 32 * kC, "the K / P and gradient passes map warp w to row or column w, lane to a channel group");
 
 // Row pitches are padded to a multiple of 4 floats so that rows can be read 16 bytes at a time.
@@ -55,7 +59,8 @@ struct BwdLayout {
     static constexpr int KM = DR + kC * LV, TM = KM + kC * LC, PM = TM + kC * LC, DPM = PM + kC * LC,
                          DTM = DPM + kC * LC, XM = DTM + kC * LC;
     static constexpr int GC = XM + kC * LC, BT = GC + DK, DB = BT + kC, DGC = DB + kC;
-    static constexpr int DGP = DGC + DK;      // [kThreads / DK][DK] partial last-row g terms
+    static constexpr int DGP = DGC + DK;      // [kThreads / DK][DK] partial last-row g terms; while
+                                              // a chunk's terms are formed, 1 / gamma_last at DGP + DK
     // staging, in bytes from its start: k, q [kC][DK] and v, dO [kC][DVH] in the input type, the
     // gate [kC][DK] fp32 (a scalar gate uses [kC]), beta [kC]
     static constexpr int ST = DGP + kThreads;
@@ -119,6 +124,7 @@ __global__ void __launch_bounds__(kThreads, 1) kda_chunk_bwd_kernel(BwdArgs b) {
     float *KM = sm + L::KM, *TM = sm + L::TM, *PM = sm + L::PM, *DPM = sm + L::DPM, *DTM = sm + L::DTM;
     float *XM = sm + L::XM, *GC = sm + L::GC, *BT = sm + L::BT, *DB = sm + L::DB, *DGC = sm + L::DGC;
     float *DGP = sm + L::DGP;
+    float *RGC = DGP + DK;         // 1 / gamma_last of the chunk while its terms are formed (fast chunks)
     uint8_t *STG = reinterpret_cast<uint8_t *>(sm + L::ST);
 
     const KdaChunkArgs &a = b.a;
@@ -203,7 +209,7 @@ __global__ void __launch_bounds__(kThreads, 1) kda_chunk_bwd_kernel(BwdArgs b) {
     // Takes chunk c0's rows from the staging area (zeros / alpha = 1 / beta = 0 past the sequence
     // end; with_q: also q and dO), starts the copies of the next chunk (pf_nr rows from pf_c0,
     // none when pf_nr = 0), and forms the decay products and the chunk matrices K, T, P.
-    auto chunk_terms = [&](int64_t c0, int nr, bool with_q, int64_t pf_c0, int pf_nr, bool pf_q) {
+    auto chunk_terms = [&](int64_t c0, int nr, bool with_q, int64_t pf_c0, int pf_nr, bool pf_q) -> bool {
         cp_async_wait_all();
         __syncthreads();                       // this chunk's staged rows are visible to all
         {
@@ -246,6 +252,7 @@ __global__ void __launch_bounds__(kThreads, 1) kda_chunk_bwd_kernel(BwdArgs b) {
                 SQ[r * LK + c] = scale * Q[r * LK + c] * g;
             }
             GC[c] = g;
+            RGC[c] = 1.f / g;
             float kp = 1.f;
 #pragma unroll
             for (int r = CH - 1; r >= 0; --r) {
@@ -254,10 +261,29 @@ __global__ void __launch_bounds__(kThreads, 1) kda_chunk_bwd_kernel(BwdArgs b) {
                 kp *= AL[r * LK + c];
             }
         }
+        const bool fast = __syncthreads_and(tid >= DK || GC[tid] >= kFastGammaMin);
+        if (fast) {
+            // K = (k gamma)(k kappa / gamma_last)^T, P = (s q gamma)(k kappa / gamma_last)^T (lower
+            // parts).  Thread: (row r, column i).
+            if (tid < CH * CH) {
+                const int r = tid / CH, i = tid % CH;
+                float sk = 0.f, sp = 0.f;
+                if (i <= r) {
+#pragma unroll 4
+                    for (int c = 0; c < DK; c += 4) {
+                        const float4 kk = ld4(KK + i * LK + c), rg = ld4(RGC + c);
+                        const float4 ki = make_float4(kk.x * rg.x, kk.y * rg.y, kk.z * rg.z, kk.w * rg.w);
+                        sk = dot4(ld4(KG + r * LK + c), ki, sk);
+                        sp = dot4(ld4(SQ + r * LK + c), ki, sp);
+                    }
+                }
+                KM[r * LC + i] = r > i ? sk : 0.f;
+                PM[r * LC + i] = r >= i ? sp : 0.f;
+            }
+        } else {
         // K and P: warp i, lane = channel group cg of 32, carries running products down the rows
         // r >= i; the 32 groups of a column are then summed by full-warp shuffles, all rows'
         // sums together (every lane of the warp takes part).
-        {
             const int i = tid >> 5, cg = tid & 31;
             constexpr int CPT = DK / 32;
             float f[CPT], sk[CH], sp[CH];
@@ -338,6 +364,7 @@ __global__ void __launch_bounds__(kThreads, 1) kda_chunk_bwd_kernel(BwdArgs b) {
             }
         }
         __syncthreads();
+        return fast;
     };
 
     // ---------------------------------------------------------------- forward: checkpoints
@@ -389,7 +416,7 @@ __global__ void __launch_bounds__(kThreads, 1) kda_chunk_bwd_kernel(BwdArgs b) {
 #pragma unroll 4
         for (int v4 = tid; v4 < DK * DVH / 4; v4 += kThreads)
             *reinterpret_cast<float4 *>(S + (4 * v4 / DVH) * LV + 4 * v4 % DVH) = ld4(src + 4 * v4);
-        chunk_terms(c0, nr, true, c0 - CH, ci > 0 ? CH : 0, true);
+        const bool fast = chunk_terms(c0, nr, true, c0 - CH, ci > 0 ? CH : 0, true);
 
         // du = P^T dO + (k kappa) dS', then dr = Diag(beta) T^T du (this half's dv rows).
         // Thread: column j, RPT rows.
@@ -509,9 +536,62 @@ __global__ void __launch_bounds__(kThreads, 1) kda_chunk_bwd_kernel(BwdArgs b) {
             DTM[r * LC + i] *= BT[r];            // dK
         }
         __syncthreads();
+        if (fast) {
+            // through D = gamma_r / gamma_i in K and P, as products: for row / column x and channel c
+            //   adk = (1 / gamma_x) sum_r (dP_rx (s q gamma)_r + dK_rx (k gamma)_r),  adg = -k_x adk,
+            //   bdq = s (gamma_x / gamma_last) sum_i dP_xi (k kappa)_i,  bdk likewise with dK,
+            //   bdg = q_x bdq + k_x bdk.
+            // Thread: rows x and x + 8, channels c .. c + 3.
+            constexpr int C4 = DK / 4;
+            if (tid < 8 * C4) {
+                const int xa = tid / C4, c = 4 * (tid % C4);
+                float4 a[2] = {}, b1[2] = {}, b2[2] = {};
+#pragma unroll
+                for (int r = 0; r < CH; ++r) {
+                    const float4 sq = ld4(SQ + r * LK + c), kg = ld4(KG + r * LK + c), kk = ld4(KK + r * LK + c);
+#pragma unroll
+                    for (int h2 = 0; h2 < 2; ++h2) {
+                        const int x = xa + 8 * h2;
+                        const float pc = DPM[r * LC + x], kc = DTM[r * LC + x], pr = DPM[x * LC + r], kr = DTM[x * LC + r];
+                        a[h2].x = fmaf(pc, sq.x, fmaf(kc, kg.x, a[h2].x));
+                        a[h2].y = fmaf(pc, sq.y, fmaf(kc, kg.y, a[h2].y));
+                        a[h2].z = fmaf(pc, sq.z, fmaf(kc, kg.z, a[h2].z));
+                        a[h2].w = fmaf(pc, sq.w, fmaf(kc, kg.w, a[h2].w));
+                        b1[h2].x = fmaf(pr, kk.x, b1[h2].x);
+                        b1[h2].y = fmaf(pr, kk.y, b1[h2].y);
+                        b1[h2].z = fmaf(pr, kk.z, b1[h2].z);
+                        b1[h2].w = fmaf(pr, kk.w, b1[h2].w);
+                        b2[h2].x = fmaf(kr, kk.x, b2[h2].x);
+                        b2[h2].y = fmaf(kr, kk.y, b2[h2].y);
+                        b2[h2].z = fmaf(kr, kk.z, b2[h2].z);
+                        b2[h2].w = fmaf(kr, kk.w, b2[h2].w);
+                    }
+                }
+                const float4 gc = ld4(GC + c);     // RGC's space is taken by the g terms by now
+                const float rgv[4] = {1.f / gc.x, 1.f / gc.y, 1.f / gc.z, 1.f / gc.w};
+#pragma unroll
+                for (int h2 = 0; h2 < 2; ++h2) {
+                    const int x = xa + 8 * h2, o = x * LK + c;
+                    const float4 ka = ld4(KA + o), ga = ld4(GA + o), kx = ld4(Kk + o), qx = ld4(Q + o);
+                    const float kav[4] = {ka.x, ka.y, ka.z, ka.w}, gav[4] = {ga.x, ga.y, ga.z, ga.w};
+                    const float kxv[4] = {kx.x, kx.y, kx.z, kx.w}, qxv[4] = {qx.x, qx.y, qx.z, qx.w};
+                    const float av[4] = {a[h2].x, a[h2].y, a[h2].z, a[h2].w};
+                    const float b1v[4] = {b1[h2].x, b1[h2].y, b1[h2].z, b1[h2].w};
+                    const float b2v[4] = {b2[h2].x, b2[h2].y, b2[h2].z, b2[h2].w};
+#pragma unroll
+                    for (int j = 0; j < 4; ++j) {
+                        const float adk = kav[j] * rgv[j] * av[j];
+                        const float gr = gav[j] * rgv[j];
+                        const float bdq = scale * gr * b1v[j], bdk = gr * b2v[j];
+                        DQ[o + j] += bdq;
+                        DKc[o + j] += adk + bdk;
+                        DG[o + j] += -kxv[j] * adk + (qxv[j] * bdq + kxv[j] * bdk);
+                    }
+                }
+            }
+        } else {
         // through D = e^{g_r - g_i} in K and P: warp x, lane = channel group cg; as column i = x
         // it walks rows r >= x, as row r = x it walks columns i <= x, each with running products.
-        {
             const int x = tid >> 5, cg = tid & 31;
             constexpr int CPT = DK / 32;
 #pragma unroll
