@@ -655,7 +655,7 @@ def roofline_entry(wl, launch_ms, hbm, peak_kind, name):
     if wl.get("bound") == "alu":
         achieved = wl["flops"] / (launch_ms / 1e3) / 1e12
         return {"bound": "alu", "achieved": achieved, "peak": FP32_PEAK_TFLOPS, "unit": "TFLOP/s",
-                "frac": achieved / FP32_PEAK_TFLOPS, "traffic": None,
+                "frac": achieved / FP32_PEAK_TFLOPS, "traffic": profiled_traffic(wl["kernel_key"], name),
                 "peak_kind": "fp32 FMA peak from the unit counts (148 SMs x 128 lanes x 2 x 1.965 GHz)",
                 "kernel": "kda_chunk_bwd_kernel + kda_chunk_bwd_reduce_kernel (one kda_chunk_bwd call)",
                 "alg_flops_per_launch": wl["flops"], "alg_bytes_per_launch": wl["bytes"],
@@ -667,7 +667,9 @@ def roofline_entry(wl, launch_ms, hbm, peak_kind, name):
             "kernel": {"chunk": "kda_chunk_intra_kernel + kda_chunk_scan_kernel "
                                 "(one kda_chunk_fwd call)",
                        "chunk_simt": "kda_chunk_simt_kernel",
-                       "decode": "kda_decode_step_kernel (one token) / kda_decode_kernel (general)"}[wl["kernel_key"]],
+                       "decode": "kda_decode_step_kernel (one token, per-channel gate) / "
+                                 "kda_decode_single_kernel (one token, other forms) / "
+                                 "kda_decode_kernel (L tokens)"}[wl["kernel_key"]],
             "alg_bytes_per_launch": wl["bytes"], "launch_ms": launch_ms}
 
 
