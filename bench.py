@@ -207,6 +207,18 @@ def profiled_traffic(kernel_key: str, workload: str):
     return float(m.group(1))
 
 
+def cpu_model() -> str:
+    """The host CPU's model name (Linux /proc/cpuinfo), recorded beside the oracle's core count."""
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    return "unknown"
+
+
 def measured_peaks():
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(path):
@@ -277,7 +289,7 @@ def cpu_baseline(inp, budget_s: float = 12.0, gpu_pair=None):
                                     tasks=tasks, nthreads=threads)
     dt = time.perf_counter() - t
     tok_heads = int(sum(lens[n] for n, _ in tasks))
-    res = {"value": tok_heads / inp.H / dt, "unit": "tokens/s", "cores": threads,
+    res = {"value": tok_heads / inp.H / dt, "unit": "tokens/s", "cores": threads, "cpu_model": cpu_model(),
            "kind": "oracle", "seconds": round(dt, 3),
            "sample": f"{n_pairs} of {inp.n_seqs * inp.H} (sequence, head) pairs, "
                      f"{tok_heads} token-heads, fp64 recurrence, {threads} threads"}
@@ -331,7 +343,7 @@ def cpu_baseline_backward(inp, dO, dSf, holder, budget_s):
                         tasks=order[:n_pairs], nthreads=threads)
     dt = time.perf_counter() - t
     res = {"value": sum(int(lens[n]) for n, _ in order[:n_pairs]) / inp.H / dt, "unit": "tokens/s",
-           "cores": threads, "kind": "oracle", "seconds": round(dt, 3),
+           "cores": threads, "cpu_model": cpu_model(), "kind": "oracle", "seconds": round(dt, 3),
            "sample": f"{n_pairs} of {inp.n_seqs * inp.H} (sequence, head) pairs, fp64 reverse mode, "
                      f"{threads} threads"}
     try:
@@ -382,7 +394,7 @@ def cpu_baseline_decode_ex(ins, S0, L, budget_s, gpu_pair):
     t = time.perf_counter()
     outs, states = oracle.recurrent(*arrs, S0, cu, tasks=order[:n_pairs], nthreads=threads)
     dt = time.perf_counter() - t
-    res = {"value": n_pairs * calls * L / H / dt, "unit": "tokens/s", "cores": threads, "kind": "oracle",
+    res = {"value": n_pairs * calls * L / H / dt, "unit": "tokens/s", "cores": threads, "cpu_model": cpu_model(), "kind": "oracle",
            "seconds": round(dt, 3),
            "sample": f"{n_pairs} of {N * H} (sequence, head) states x {calls} calls of {L} tokens, "
                      f"fp64 recurrence, {threads} threads"}
@@ -412,7 +424,7 @@ def cpu_baseline_decode(ins, S0, budget_s: float = 12.0, gpu_pair=None):
     outs, states = oracle.recurrent(*arrs, S0, cu, tasks=order[:n_pairs], nthreads=threads)
     dt = time.perf_counter() - t
     # a decode token is one sequence's step over all H heads
-    res = {"value": n_pairs * steps / H / dt, "unit": "tokens/s", "cores": threads,
+    res = {"value": n_pairs * steps / H / dt, "unit": "tokens/s", "cores": threads, "cpu_model": cpu_model(),
            "kind": "oracle", "seconds": round(dt, 3),
            "sample": f"{n_pairs} of {N * H} (sequence, head) states x {steps} steps, "
                      f"fp64 recurrence, {threads} threads"}
@@ -792,12 +804,13 @@ def decode_pairs(dev_in, S0, device, kda_decode_step):
     return gpu_pair
 
 
-def run_e2e(args, name, device, stream, rank):
+def run_e2e(args, name, device, stream, rank, return_outputs=False):
     """The same metric through the public call with pinned host buffers: every step copies its
     inputs host -> device, makes the call and copies its results back, all inside the timed
     region.  The N sequences go in up to four groups on three streams (copies in, the calls,
     copies out), so a group's results travel back while the next group's inputs travel in and
-    another group is computed: the host link carries both directions at once."""
+    another group is computed: the host link carries both directions at once.  With
+    ``return_outputs`` the host buffers of the last step's results come back too (for tests)."""
     import torch
     from gated_delta_rule_119_b200 import kda_chunk_fwd, kda_decode_step
     w = WORKLOADS[name]
@@ -884,11 +897,12 @@ def run_e2e(args, name, device, stream, rank):
     torch.cuda.synchronize(device)
     ms = reduce_max(ev0.elapsed_time(ev1) / steps, device)
     world = int(os.environ.get("WORLD_SIZE", 1))
-    return {"value": units * world / (ms / 1e3), "unit": "tokens/s", "ms_per_step": ms,
-            "steps": steps, "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
-            "path": f"pinned host -> kda_* public call -> pinned host, the sequences in {P} groups on "
-                    "three streams (copies in, calls, copies out overlapping)"
-                    + (" (decode state resident in HBM)" if name == "decode" else "")}
+    res = {"value": units * world / (ms / 1e3), "unit": "tokens/s", "ms_per_step": ms,
+           "steps": steps, "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
+           "path": f"pinned host -> kda_* public call -> pinned host, the sequences in {P} groups on "
+                   "three streams (copies in, calls, copies out overlapping)"
+                   + (" (decode state resident in HBM)" if name == "decode" else "")}
+    return (res, host, out_host, S_host) if return_outputs else res
 
 
 def run_reference(args, rank, world):
@@ -915,11 +929,29 @@ def run_reference(args, rank, world):
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
             "data": "synthetic (seeded numpy; see inputs.py recipe)",
             "config": workload_config(name, None, 1),
-            "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": samples[-1]["cores"],
+            "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": samples[-1]["cores"], "cpu_model": cpu_model(),
                              "kind": "oracle", "sample": samples[-1]["sample"]},
             "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0,
                     "d2h_bytes_per_step": 0},
             "gpu_launches": 0}
+
+
+def profile_bwd_small():
+    """Three kda_chunk_bwd calls on B=4 T=512 H=16 dk=dv=128 bf16: the prefill_bwd workload's
+    CTAs (one per (sequence, head, d_v half)) with an eighth of its chunks, a case small enough
+    for a full ncu capture."""
+    import torch
+    from gated_delta_rule_119_b200 import kda_chunk_bwd
+    d = to_torch(make_inputs(4, 512, 16, 128, 128, "bf16", 3), "cuda")
+    g = torch.Generator(device="cpu").manual_seed(5)
+    dO = torch.randn(d["v"].shape, generator=g).to("cuda").to(d["q"].dtype)
+    for _ in range(3):
+        r = kda_chunk_bwd(d["q"], d["k"], d["v"], d["log_alpha"], d["beta"], dO, d["S0"], d["cu_seqlens"])
+    torch.cuda.synchronize()
+    print("ok", float(r["dq"].float().abs().max()), flush=True)
+
+
+PROFILE_CASES = {"bwd_small": profile_bwd_small}
 
 
 def main(argv=None):
@@ -945,7 +977,12 @@ def main(argv=None):
                     help="other workloads measured in the same process at N=1 (comma list; "
                          "empty for none)")
     ap.add_argument("--workload-parity-budget", type=float, default=3.0)
+    ap.add_argument("--profile-case", choices=sorted(PROFILE_CASES),
+                    help="only run the named small case a few times (for ncu captures) and exit")
     args = ap.parse_args(argv)
+    if args.profile_case:
+        PROFILE_CASES[args.profile_case]()
+        return 0
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
     rank, local_rank, world = dist_env()
