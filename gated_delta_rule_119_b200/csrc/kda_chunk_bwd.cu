@@ -39,6 +39,7 @@ constexpr int kC = 16;
 // [1, e^80] or [e^-80, 1]: K, P and their gradients through D become plain small products.
 constexpr float kFastGammaMin = 1.8048513e-35f;   // e^-80
 static_assert(kThreads == 32 * kC, "the K / P and gradient passes map warp w to row or column w, lane to a channel group");
+static_assert(2 * 128 + 128 <= kThreads - kC, "gradient products, rowsum and dbeta on separate threads");
 
 // Row pitches are padded to a multiple of 4 floats so that rows can be read 16 bytes at a time.
 // ES is the input element size; the staging area at the end holds the next chunk's raw inputs
@@ -337,24 +338,28 @@ __global__ void __launch_bounds__(kThreads, 1) kda_chunk_bwd_kernel(BwdArgs b) {
             }
         }
         __syncthreads();
-        // r = v - (k gamma) S;  then u = T Diag(beta) r.  Thread: column j, RPT rows.
+        // r = v - (k gamma) S (thread: column j, 4 rows, so each state value feeds 4 rows); then
+        // u = T Diag(beta) r (thread: column j, RPT rows).
         {
-            const int j = tid % DVH, r0 = (tid / DVH) * RPT;
-            float acc[RPT];
+            if (tid < 4 * DVH) {
+                const int j = tid % DVH, r0 = (tid / DVH) * 4;
+                float acc[4];
 #pragma unroll
-            for (int t = 0; t < RPT; ++t) acc[t] = V[(r0 + t) * LV + j];
-            for (int c = 0; c < DK; c += 4) {
-                const float4 s4 = make_float4(S[c * LV + j], S[(c + 1) * LV + j], S[(c + 2) * LV + j],
-                                              S[(c + 3) * LV + j]);
+                for (int t = 0; t < 4; ++t) acc[t] = V[(r0 + t) * LV + j];
+                for (int c = 0; c < DK; c += 4) {
+                    const float4 s4 = make_float4(S[c * LV + j], S[(c + 1) * LV + j], S[(c + 2) * LV + j],
+                                                  S[(c + 3) * LV + j]);
 #pragma unroll
-                for (int t = 0; t < RPT; ++t) {
-                    const float4 kg = ld4(KG + (r0 + t) * LK + c);
-                    acc[t] = dot4(make_float4(-kg.x, -kg.y, -kg.z, -kg.w), s4, acc[t]);
+                    for (int t = 0; t < 4; ++t) {
+                        const float4 kg = ld4(KG + (r0 + t) * LK + c);
+                        acc[t] = dot4(make_float4(-kg.x, -kg.y, -kg.z, -kg.w), s4, acc[t]);
+                    }
                 }
-            }
 #pragma unroll
-            for (int t = 0; t < RPT; ++t) R[(r0 + t) * LV + j] = acc[t];
+                for (int t = 0; t < 4; ++t) R[(r0 + t) * LV + j] = acc[t];
+            }
             __syncthreads();
+            const int j = tid % DVH, r0 = (tid / DVH) * RPT;
 #pragma unroll
             for (int t = 0; t < RPT; ++t) {
                 const int r = r0 + t;
@@ -421,24 +426,27 @@ __global__ void __launch_bounds__(kThreads, 1) kda_chunk_bwd_kernel(BwdArgs b) {
         // du = P^T dO + (k kappa) dS', then dr = Diag(beta) T^T du (this half's dv rows).
         // Thread: column j, RPT rows.
         {
-            const int j = tid % DVH, i0 = (tid / DVH) * RPT;
-            float acc[RPT];
+            if (tid < 4 * DVH) {                   // du: thread column j, 4 rows
+                const int j = tid % DVH, i0 = (tid / DVH) * 4;
+                float acc[4];
 #pragma unroll
-            for (int t = 0; t < RPT; ++t) {
-                const int i = i0 + t;
-                float a0 = 0.f;
-                for (int r = i; r < CH; ++r) a0 = fmaf(PM[r * LC + i], DO[r * LV + j], a0);
-                acc[t] = a0;
+                for (int t = 0; t < 4; ++t) {
+                    const int i = i0 + t;
+                    float a0 = 0.f;
+                    for (int r = i; r < CH; ++r) a0 = fmaf(PM[r * LC + i], DO[r * LV + j], a0);
+                    acc[t] = a0;
+                }
+                for (int c = 0; c < DK; c += 4) {
+                    const float4 d4 = make_float4(DS[c * LV + j], DS[(c + 1) * LV + j], DS[(c + 2) * LV + j],
+                                                  DS[(c + 3) * LV + j]);
+#pragma unroll
+                    for (int t = 0; t < 4; ++t) acc[t] = dot4(ld4(KK + (i0 + t) * LK + c), d4, acc[t]);
+                }
+#pragma unroll
+                for (int t = 0; t < 4; ++t) DU[(i0 + t) * LV + j] = acc[t];
             }
-            for (int c = 0; c < DK; c += 4) {
-                const float4 d4 = make_float4(DS[c * LV + j], DS[(c + 1) * LV + j], DS[(c + 2) * LV + j],
-                                              DS[(c + 3) * LV + j]);
-#pragma unroll
-                for (int t = 0; t < RPT; ++t) acc[t] = dot4(ld4(KK + (i0 + t) * LK + c), d4, acc[t]);
-            }
-#pragma unroll
-            for (int t = 0; t < RPT; ++t) DU[(i0 + t) * LV + j] = acc[t];
             __syncthreads();
+            const int j = tid % DVH, i0 = (tid / DVH) * RPT;   // dr: thread column j, RPT rows
 #pragma unroll
             for (int t = 0; t < RPT; ++t) {
                 const int i = i0 + t;
@@ -464,48 +472,67 @@ __global__ void __launch_bounds__(kThreads, 1) kda_chunk_bwd_kernel(BwdArgs b) {
         }
         __syncthreads();
         // the decay-weighted elementwise terms: d(s q gamma) = dO S^T, d(k gamma) = -dr S^T,
-        // d(k kappa) = u dS'^T, and the last row's g terms.  Thread: channel c, R7 rows.
+        // d(k kappa) = u dS'^T, and the last row's g terms.  Thread: channels c and c + DK / 2, 4 rows
+        // (each broadcast row of dO, dr, u feeds both channels); beside them other warps form
+        // gamma_last rowsum(dS' * S) and dbeta from T' = T Diag(beta).
         {
-            const int c = tid % DK, g7 = tid / DK, r0 = g7 * R7;
-            float dsq[R7], dkg[R7], dkk[R7];
+            constexpr int NTH = 2 * DK;
+            if (tid < NTH) {
+                const int cp = tid % (DK / 2), g4 = tid / (DK / 2), r0 = 4 * g4;
+                const int cc[2] = {cp, cp + DK / 2};
+                float dsq[2][4], dkg[2][4], dkk[2][4];
 #pragma unroll
-            for (int t = 0; t < R7; ++t) dsq[t] = dkg[t] = dkk[t] = 0.f;
-            float gl = 0.f;
-            for (int j = 0; j < DVH; j += 4) {
-                const float4 s4 = ld4(S + c * LV + j), d4 = ld4(DS + c * LV + j);
-                if (g7 == 0) gl = dot4(d4, s4, gl);
+                for (int hh = 0; hh < 2; ++hh)
 #pragma unroll
-                for (int t = 0; t < R7; ++t) {
-                    const int r = r0 + t;
-                    const float4 dr = ld4(DR + r * LV + j);
-                    dsq[t] = dot4(ld4(DO + r * LV + j), s4, dsq[t]);
-                    dkg[t] = dot4(make_float4(-dr.x, -dr.y, -dr.z, -dr.w), s4, dkg[t]);
-                    dkk[t] = dot4(ld4(U + r * LV + j), d4, dkk[t]);
+                    for (int t = 0; t < 4; ++t) dsq[hh][t] = dkg[hh][t] = dkk[hh][t] = 0.f;
+                for (int j = 0; j < DVH; j += 4) {
+                    const float4 s0 = ld4(S + cc[0] * LV + j), s1 = ld4(S + cc[1] * LV + j);
+                    const float4 d0 = ld4(DS + cc[0] * LV + j), d1 = ld4(DS + cc[1] * LV + j);
+#pragma unroll
+                    for (int t = 0; t < 4; ++t) {
+                        const int r = r0 + t;
+                        const float4 o4 = ld4(DO + r * LV + j), dr = ld4(DR + r * LV + j), u4 = ld4(U + r * LV + j);
+                        const float4 nd = make_float4(-dr.x, -dr.y, -dr.z, -dr.w);
+                        dsq[0][t] = dot4(o4, s0, dsq[0][t]);
+                        dsq[1][t] = dot4(o4, s1, dsq[1][t]);
+                        dkg[0][t] = dot4(nd, s0, dkg[0][t]);
+                        dkg[1][t] = dot4(nd, s1, dkg[1][t]);
+                        dkk[0][t] = dot4(u4, d0, dkk[0][t]);
+                        dkk[1][t] = dot4(u4, d1, dkk[1][t]);
+                    }
                 }
-            }
-            float kkp = 0.f;
 #pragma unroll
-            for (int t = 0; t < R7; ++t) {
-                const int r = r0 + t;
-                DQ[r * LK + c] = scale * GA[r * LK + c] * dsq[t];
-                DKc[r * LK + c] = GA[r * LK + c] * dkg[t] + KA[r * LK + c] * dkk[t];
-                DG[r * LK + c] = dsq[t] * SQ[r * LK + c] + dkg[t] * KG[r * LK + c] - dkk[t] * KK[r * LK + c];
-                kkp = fmaf(dkk[t], KK[r * LK + c], kkp);
+                for (int hh = 0; hh < 2; ++hh) {
+                    const int c = cc[hh];
+                    float kkp = 0.f;
+#pragma unroll
+                    for (int t = 0; t < 4; ++t) {
+                        const int o = (r0 + t) * LK + c;
+                        DQ[o] = scale * GA[o] * dsq[hh][t];
+                        DKc[o] = GA[o] * dkg[hh][t] + KA[o] * dkk[hh][t];
+                        DG[o] = dsq[hh][t] * SQ[o] + dkg[hh][t] * KG[o] - dkk[hh][t] * KK[o];
+                        kkp = fmaf(dkk[hh][t], KK[o], kkp);
+                    }
+                    DGP[g4 * DK + c] = kkp;           // summed over the 4 row groups below, in order
+                }
+            } else if (tid < NTH + DK) {
+                const int c = tid - NTH;
+                float gl = 0.f;
+                for (int j = 0; j < DVH; j += 4) gl = dot4(ld4(DS + c * LV + j), ld4(S + c * LV + j), gl);
+                DGC[c] = GC[c] * gl;
             }
-            DGP[g7 * DK + c] = kkp;
-            if (g7 == 0) DGC[c] = GC[c] * gl;   // the partial terms are added below, in group order
-        }
-        // dbeta from T' = T Diag(beta); dT = dT' Diag(beta); X = dT T^T
-        if (tid < CH) {
-            const int i = tid;
-            float acc = 0.f;
-            for (int r = i; r < CH; ++r) acc = fmaf(DTM[r * LC + i], TM[r * LC + i], acc);
-            DB[i] = acc;
+            if (tid >= kThreads - CH) {
+                const int i = tid - (kThreads - CH);
+                float acc = 0.f;
+                for (int r = i; r < CH; ++r) acc = fmaf(DTM[r * LC + i], TM[r * LC + i], acc);
+                DB[i] = acc;
+            }
         }
         __syncthreads();
+        // dT = dT' Diag(beta); X = dT T^T; the last row's g terms summed
         for (int c = tid; c < DK; c += kThreads) {
             float acc = DGC[c];
-            for (int g = 0; g < kThreads / DK; ++g) acc += DGP[g * DK + c];
+            for (int g = 0; g < CH / 4; ++g) acc += DGP[g * DK + c];
             DGC[c] = acc;                     // both go to the last row's g
         }
         for (int idx = tid; idx < CH * CH; idx += kThreads) {
