@@ -117,6 +117,8 @@ __global__ void __launch_bounds__(kThreads, 1) kda_chunk_bwd_kernel(BwdArgs b) {
     constexpr int R7 = kC * DK / kThreads;     // rows per thread of the [C][dk] products
     static_assert(RPT >= 1 && (CPT % 4 == 0 || CPT < 4) && R7 >= 1 && DK % 32 == 0 && DVH % 4 == 0,
                   "backward tiling");
+    constexpr int NTU = (DVH / 2) * (DK / 16);   // threads of the state updates (2 columns x 16 rows)
+    static_assert(NTU <= kThreads, "state update tiling");
     extern __shared__ float sm[];
     float *Q = sm + L::Q, *Kk = sm + L::Kk, *AL = sm + L::AL, *GA = sm + L::GA, *KA = sm + L::KA;
     float *KG = sm + L::KG, *SQ = sm + L::SQ, *KK = sm + L::KK, *DQ = sm + L::DQ, *DKc = sm + L::DKc;
@@ -385,30 +387,32 @@ __global__ void __launch_bounds__(kThreads, 1) kda_chunk_bwd_kernel(BwdArgs b) {
         // next: chunk ci + 1, or after the last one the backward pass's first chunk (the last)
         const int nx = ci + 1 < nch ? ci + 1 : nch - 1;
         chunk_terms(c0, nr, false, t0 + (int64_t)nx * CH, chunk_rows(nx), ci + 1 >= nch);
-        // S <- Diag(gamma_last) S + (k kappa)^T u, in place.  Thread: column j, CPT rows.
-        {
-            const int j = tid % DVH, c0 = (tid / DVH) * CPT;
-            float acc[CPT];
+        // S <- Diag(gamma_last) S + (k kappa)^T u, in place.  Thread: columns j, j + 1 and 16 rows
+        // (each broadcast (k kappa) value feeds both columns).
+        if (tid < NTU) {
+            const int j = 2 * (tid % (DVH / 2)), c0 = (tid / (DVH / 2)) * 16;
+            float2 acc[16];
 #pragma unroll
-            for (int t = 0; t < CPT; ++t) acc[t] = GC[c0 + t] * S[(c0 + t) * LV + j];
+            for (int t = 0; t < 16; ++t) {
+                const float g = GC[c0 + t];
+                const float2 x = *reinterpret_cast<const float2 *>(S + (c0 + t) * LV + j);
+                acc[t] = make_float2(g * x.x, g * x.y);
+            }
             for (int r = 0; r < CH; ++r) {
-                const float u = U[r * LV + j];
-                if constexpr (CPT % 4 == 0) {
+                const float2 u = *reinterpret_cast<const float2 *>(U + r * LV + j);
 #pragma unroll
-                    for (int t = 0; t < CPT; t += 4) {
-                        const float4 kk = ld4(KK + r * LK + c0 + t);
-                        acc[t] = fmaf(kk.x, u, acc[t]);
-                        acc[t + 1] = fmaf(kk.y, u, acc[t + 1]);
-                        acc[t + 2] = fmaf(kk.z, u, acc[t + 2]);
-                        acc[t + 3] = fmaf(kk.w, u, acc[t + 3]);
+                for (int t = 0; t < 16; t += 4) {
+                    const float4 kk = ld4(KK + r * LK + c0 + t);
+                    const float kv[4] = {kk.x, kk.y, kk.z, kk.w};
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        acc[t + e].x = fmaf(kv[e], u.x, acc[t + e].x);
+                        acc[t + e].y = fmaf(kv[e], u.y, acc[t + e].y);
                     }
-                } else {
-#pragma unroll
-                    for (int t = 0; t < CPT; ++t) acc[t] = fmaf(KK[r * LK + c0 + t], u, acc[t]);
                 }
             }
 #pragma unroll
-            for (int t = 0; t < CPT; ++t) S[(c0 + t) * LV + j] = acc[t];
+            for (int t = 0; t < 16; ++t) *reinterpret_cast<float2 *>(S + (c0 + t) * LV + j) = acc[t];
         }
         __syncthreads();
     }
@@ -664,31 +668,32 @@ __global__ void __launch_bounds__(kThreads, 1) kda_chunk_bwd_kernel(BwdArgs b) {
         }
         if (tid < nr) b.part[part_index(b, split, (size_t)(c0 + tid) * H + h, DK) + 3 * DK] = DB[tid];
         // dS for the previous chunk, in place: (s q gamma)^T dO + Diag(gamma_last) dS' - (k gamma)^T dr.
-        // Thread: column j, CPT rows.
-        {
-            const int j = tid % DVH, cb = (tid / DVH) * CPT;
-            float acc[CPT];
+        // Thread: columns j, j + 1 and 16 rows.
+        if (tid < NTU) {
+            const int j = 2 * (tid % (DVH / 2)), cb = (tid / (DVH / 2)) * 16;
+            float2 acc[16];
 #pragma unroll
-            for (int t = 0; t < CPT; ++t) acc[t] = GC[cb + t] * DS[(cb + t) * LV + j];
+            for (int t = 0; t < 16; ++t) {
+                const float g = GC[cb + t];
+                const float2 x = *reinterpret_cast<const float2 *>(DS + (cb + t) * LV + j);
+                acc[t] = make_float2(g * x.x, g * x.y);
+            }
             for (int r = 0; r < CH; ++r) {
-                const float d = DO[r * LV + j], e = DR[r * LV + j];
-                if constexpr (CPT % 4 == 0) {
+                const float2 d = *reinterpret_cast<const float2 *>(DO + r * LV + j);
+                const float2 e2 = *reinterpret_cast<const float2 *>(DR + r * LV + j);
 #pragma unroll
-                    for (int t = 0; t < CPT; t += 4) {
-                        const float4 sq = ld4(SQ + r * LK + cb + t), kg = ld4(KG + r * LK + cb + t);
-                        acc[t] = fmaf(sq.x, d, fmaf(-kg.x, e, acc[t]));
-                        acc[t + 1] = fmaf(sq.y, d, fmaf(-kg.y, e, acc[t + 1]));
-                        acc[t + 2] = fmaf(sq.z, d, fmaf(-kg.z, e, acc[t + 2]));
-                        acc[t + 3] = fmaf(sq.w, d, fmaf(-kg.w, e, acc[t + 3]));
+                for (int t = 0; t < 16; t += 4) {
+                    const float4 sq = ld4(SQ + r * LK + cb + t), kg = ld4(KG + r * LK + cb + t);
+                    const float sv[4] = {sq.x, sq.y, sq.z, sq.w}, gv[4] = {kg.x, kg.y, kg.z, kg.w};
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        acc[t + e].x = fmaf(sv[e], d.x, fmaf(-gv[e], e2.x, acc[t + e].x));
+                        acc[t + e].y = fmaf(sv[e], d.y, fmaf(-gv[e], e2.y, acc[t + e].y));
                     }
-                } else {
-#pragma unroll
-                    for (int t = 0; t < CPT; ++t)
-                        acc[t] = fmaf(SQ[r * LK + cb + t], d, fmaf(-KG[r * LK + cb + t], e, acc[t]));
                 }
             }
 #pragma unroll
-            for (int t = 0; t < CPT; ++t) DS[(cb + t) * LV + j] = acc[t];
+            for (int t = 0; t < 16; ++t) *reinterpret_cast<float2 *>(DS + (cb + t) * LV + j) = acc[t];
         }
         __syncthreads();
     }
