@@ -436,27 +436,28 @@ __global__ void __launch_bounds__(NTHR, 2)
         // k e^-g / [I; P], left s q in place of q (each thread rewrites the elements it read)
         uint8_t *sKL = sm + I_AM, *sKR = sm + I_KC;
         if (fast) {
-            float l0 = 1.f, l1 = 1.f;
+            // both channels at once on packed fp32 pairs (each lane rounded as the plain product)
+            float2 l = make_float2(1.f, 1.f);
+            const float2 sc2 = make_float2(scale, scale);
 #pragma unroll
             for (int rr = 0; rr < 16; ++rr) {
                 const int r = 16 * eb + rr;
-                l0 *= la[rr].x;
-                l1 *= la[rr].y;
+                l = __fmul2_rn(l, la[rr]);
                 const float2 kv = row_scaled<NORM>(unpack_bf16(kr2[rr]), sRk, r);
                 const float2 qv = row_scaled<NORM>(unpack_bf16(r < nr ? *(const uint32_t *)(sQ + rm_sw(r, c2)) : 0u), sRq, r);
-                const float g0 = gpre.x * l0, g1 = gpre.y * l1;
-                *(uint32_t *)(sKQ + col_kq + sw128(r, c2 & 63)) = pack_bf16(kv.x * g0, kv.y * g1);
-                *(uint32_t *)(sKQ + col_kq + sw128(64 + r, c2 & 63)) = pack_bf16(scale * qv.x * g0, scale * qv.y * g1);
+                const float2 g = __fmul2_rn(gpre, l);
+                const float2 kg = __fmul2_rn(kv, g), qg = __fmul2_rn(__fmul2_rn(sc2, qv), g);
+                *(uint32_t *)(sKQ + col_kq + sw128(r, c2 & 63)) = pack_bf16(kg.x, kg.y);
+                *(uint32_t *)(sKQ + col_kq + sw128(64 + r, c2 & 63)) = pack_bf16(qg.x, qg.y);
             }
-            float g0 = 1.f, g1 = 1.f;
+            float2 g = make_float2(1.f, 1.f);
 #pragma unroll
             for (int rr = 15; rr >= 0; --rr) {
                 const int r = 16 * eb + rr;
                 const float2 kv = row_scaled<NORM>(unpack_bf16(kr2[rr]), sRk, r);
-                *(uint32_t *)(sKC + col_kc + sw128(r, c2 & 63)) =
-                    pack_bf16(kv.x * (g0 * ksuf.x), kv.y * (g1 * ksuf.y));
-                g0 *= la[rr].x;
-                g1 *= la[rr].y;
+                const float2 kk = __fmul2_rn(kv, __fmul2_rn(g, ksuf));
+                *(uint32_t *)(sKC + col_kc + sw128(r, c2 & 63)) = pack_bf16(kk.x, kk.y);
+                g = __fmul2_rn(g, la[rr]);
             }
         } else {
             // The rescaled factors rho * (prefix product) and rho * (suffix product) are carried
