@@ -78,7 +78,8 @@ struct BwdArgs {
     const float *dS_final;          // [N, H, dk, dv] or NULL
     void *dv_out;                   // [T_total, H, dv] dtype
     float *dS0;                     // [N, H, dk, dv] or NULL
-    float *ckpt;                    // checkpoints: [max_chunks][H][nsplit] blocks of dk x dvh
+    float *ckpt;                    // checkpoints: [max_chunks][H][nsplit] blocks of (dk + 2 kC) x dvh:
+                                    // the chunk-start state, then the chunk's r and u
     float *part;                    // shares: [nsplit][T_total][H] x (3 dk + 1): dq, dk, dla, dbeta
     int64_t max_chunks;             // ceil(T_total / 16) + N with cu_seqlens, N ceil(T / 16) without
     int nsplit;
@@ -163,7 +164,12 @@ __global__ void __launch_bounds__(kThreads, 1) kda_chunk_bwd_kernel(BwdArgs b) {
     if (nch64 > b.max_chunks - base) nch64 = b.max_chunks - base;
     const int nch = (int)nch64;
     auto ckpt_block = [&](int ci) {
-        return b.ckpt + (((size_t)(base + ci) * H + h) * b.nsplit + split) * (size_t)DK * DVH;
+        return b.ckpt + (((size_t)(base + ci) * H + h) * b.nsplit + split) * (size_t)(DK + 2 * CH) * DVH;
+    };
+    // Copies rows of `rows` x DVH floats (packed, from global) into a padded shared array.
+    auto copy_in = [&](float *dst, const float *src, int rows) {
+        for (int q = tid; q < rows * DVH / 4; q += kThreads)
+            cp_async16(dst + (4 * q / DVH) * LV + 4 * q % DVH, src + 4 * q);
     };
     const size_t sbase = (size_t)pair * DK * dv;
 
@@ -212,7 +218,8 @@ __global__ void __launch_bounds__(kThreads, 1) kda_chunk_bwd_kernel(BwdArgs b) {
     // Takes chunk c0's rows from the staging area (zeros / alpha = 1 / beta = 0 past the sequence
     // end; with_q: also q and dO), starts the copies of the next chunk (pf_nr rows from pf_c0,
     // none when pf_nr = 0), and forms the decay products and the chunk matrices K, T, P.
-    auto chunk_terms = [&](int64_t c0, int nr, bool with_q, int64_t pf_c0, int pf_nr, bool pf_q) -> bool {
+    auto chunk_terms = [&](int64_t c0, int nr, bool with_q, int64_t pf_c0, int pf_nr, bool pf_q,
+                           bool form_ru) -> bool {
         cp_async_wait_all();
         __syncthreads();                       // this chunk's staged rows are visible to all
         {
@@ -341,8 +348,9 @@ __global__ void __launch_bounds__(kThreads, 1) kda_chunk_bwd_kernel(BwdArgs b) {
         }
         __syncthreads();
         // r = v - (k gamma) S (thread: column j, 4 rows, so each state value feeds 4 rows); then
-        // u = T Diag(beta) r (thread: column j, RPT rows).
-        {
+        // u = T Diag(beta) r (thread: column j, RPT rows).  The backward pass finds both in place
+        // (the forward pass stored them with the checkpoint).
+        if (form_ru) {
             if (tid < 4 * DVH) {
                 const int j = tid % DVH, r0 = (tid / DVH) * 4;
                 float acc[4];
@@ -386,7 +394,15 @@ __global__ void __launch_bounds__(kThreads, 1) kda_chunk_bwd_kernel(BwdArgs b) {
             *reinterpret_cast<float4 *>(dst + 4 * v4) = ld4(S + (4 * v4 / DVH) * LV + 4 * v4 % DVH);
         // next: chunk ci + 1, or after the last one the backward pass's first chunk (the last)
         const int nx = ci + 1 < nch ? ci + 1 : nch - 1;
-        chunk_terms(c0, nr, false, t0 + (int64_t)nx * CH, chunk_rows(nx), ci + 1 >= nch);
+        chunk_terms(c0, nr, false, t0 + (int64_t)nx * CH, chunk_rows(nx), ci + 1 >= nch, true);
+        {   // the chunk's r and u beside its checkpoint, for the backward pass
+            float *ru = dst + DK * DVH;
+            for (int q = tid; q < 2 * CH * DVH / 4; q += kThreads) {
+                const int row = 4 * q / DVH, j = 4 * q % DVH;
+                const float *from = row < CH ? R + row * LV + j : U + (row - CH) * LV + j;
+                *reinterpret_cast<float4 *>(ru + 4 * q) = ld4(from);
+            }
+        }
         // S <- Diag(gamma_last) S + (k kappa)^T u, in place.  Thread: columns j, j + 1 and 16 rows
         // (each broadcast (k kappa) value feeds both columns).
         if (tid < NTU) {
@@ -418,14 +434,17 @@ __global__ void __launch_bounds__(kThreads, 1) kda_chunk_bwd_kernel(BwdArgs b) {
     }
 
     // ---------------------------------------------------------------- backward
+    // Each chunk's checkpoint, r and u arrive by cp.async: the last chunk's checkpoint now (its r
+    // and u are still in place from the forward pass), every earlier chunk's once the chunk after
+    // it no longer reads S, R and U (below, after the gradient products).
+    if (nch > 0) {
+        copy_in(S, ckpt_block(nch - 1), DK);
+        cp_async_commit();
+    }
     for (int ci = nch - 1; ci >= 0; --ci) {
         const int64_t c0 = t0 + (int64_t)ci * CH;
         const int nr = (int)(t1 - c0 < CH ? t1 - c0 : CH);
-        const float *src = ckpt_block(ci);
-#pragma unroll 4
-        for (int v4 = tid; v4 < DK * DVH / 4; v4 += kThreads)
-            *reinterpret_cast<float4 *>(S + (4 * v4 / DVH) * LV + 4 * v4 % DVH) = ld4(src + 4 * v4);
-        const bool fast = chunk_terms(c0, nr, true, c0 - CH, ci > 0 ? CH : 0, true);
+        const bool fast = chunk_terms(c0, nr, true, c0 - CH, ci > 0 ? CH : 0, true, false);
 
         // du = P^T dO + (k kappa) dS', then dr = Diag(beta) T^T du (this half's dv rows).
         // Thread: column j, RPT rows.
@@ -533,6 +552,13 @@ __global__ void __launch_bounds__(kThreads, 1) kda_chunk_bwd_kernel(BwdArgs b) {
             }
         }
         __syncthreads();
+        if (ci > 0) {                          // S, R and U are not read again for this chunk
+            const float *src = ckpt_block(ci - 1);
+            copy_in(S, src, DK);
+            copy_in(R, src + DK * DVH, CH);
+            copy_in(U, src + (DK + CH) * DVH, CH);
+            cp_async_commit();
+        }
         // dT = dT' Diag(beta); X = dT T^T; the last row's g terms summed
         for (int c = tid; c < DK; c += kThreads) {
             float acc = DGC[c];
@@ -788,7 +814,7 @@ int64_t bwd_max_chunks(const KdaChunkArgs &a) {
 
 size_t kda_chunk_bwd_workspace_bytes(const KdaChunkArgs &a) {
     const int nsplit = a.dv > 64 ? a.dv / 64 : 1, dvh = a.dv / nsplit;
-    const size_t ck = (size_t)bwd_max_chunks(a) * a.H * nsplit * a.dk * dvh * sizeof(float);
+    const size_t ck = (size_t)bwd_max_chunks(a) * a.H * nsplit * (a.dk + 2 * kC) * dvh * sizeof(float);
     const size_t part = (size_t)nsplit * a.T_total * a.H * (3 * (size_t)a.dk + 1) * sizeof(float);
     return ((ck + 255) & ~(size_t)255) + part;
 }
@@ -805,7 +831,7 @@ cudaError_t kda_launch_chunk_bwd(const KdaChunkArgs &a, int dtype, const void *d
     b.nsplit = a.dv > 64 ? a.dv / 64 : 1;
     const int dvh = a.dv / b.nsplit;
     b.max_chunks = bwd_max_chunks(a);
-    const size_t ck = (size_t)b.max_chunks * a.H * b.nsplit * a.dk * dvh * sizeof(float);
+    const size_t ck = (size_t)b.max_chunks * a.H * b.nsplit * (a.dk + 2 * kC) * dvh * sizeof(float);
     b.ckpt = static_cast<float *>(ws);
     b.part = reinterpret_cast<float *>(static_cast<char *>(ws) + ((ck + 255) & ~(size_t)255));
     return dtype == 0 ? run<float>(b, dq, dk, dgate, dbeta, stream) : run<__nv_bfloat16>(b, dq, dk, dgate, dbeta, stream);
