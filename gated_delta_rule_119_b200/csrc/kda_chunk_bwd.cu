@@ -39,7 +39,8 @@ constexpr int kC = 16;
 // [1, e^80] or [e^-80, 1]: K, P and their gradients through D become plain small products.
 constexpr float kFastGammaMin = 1.8048513e-35f;   // e^-80
 static_assert(kThreads == 32 * kC, "the K / P and gradient passes map warp w to row or column w, lane to a channel group");
-static_assert(2 * 128 + 128 <= kThreads - kC, "gradient products, rowsum and dbeta on separate threads");
+static_assert(2 * 128 + 128 < kThreads - kC, "gradient products, rowsum, X and dbeta on separate threads");
+static_assert(kC * kC <= kThreads && kC == 16, "dA: one thread per entry, a row per half-warp");
 
 // Row pitches are padded to a multiple of 4 floats so that rows can be read 16 bytes at a time.
 // ES is the input element size; the staging area at the end holds the next chunk's raw inputs
@@ -549,6 +550,14 @@ __global__ void __launch_bounds__(kThreads, 1) kda_chunk_bwd_kernel(BwdArgs b) {
                 float acc = 0.f;
                 for (int r = i; r < CH; ++r) acc = fmaf(DTM[r * LC + i], TM[r * LC + i], acc);
                 DB[i] = acc;
+            } else if (tid >= NTH + DK) {        // X = dT' Diag(beta) T^T
+                for (int idx = tid - (NTH + DK); idx < CH * CH; idx += kThreads - CH - NTH - DK) {
+                    const int r = idx / CH, m = idx % CH;
+                    float acc = 0.f;
+                    for (int i = 0; i <= (r < m ? r : m); ++i)
+                        acc = fmaf(DTM[r * LC + i] * BT[i], TM[m * LC + i], acc);
+                    XM[r * LC + m] = acc;
+                }
             }
         }
         __syncthreads();
@@ -559,38 +568,25 @@ __global__ void __launch_bounds__(kThreads, 1) kda_chunk_bwd_kernel(BwdArgs b) {
             copy_in(U, src + (DK + CH) * DVH, CH);
             cp_async_commit();
         }
-        // dT = dT' Diag(beta); X = dT T^T; the last row's g terms summed
+        // The last row's g terms summed; dA = strict-lower(-T^T X) (X = dT T^T, dT = dT' Diag(beta),
+        // formed beside the gradient products), dbeta_p += sum_m dA_pm K_pm (the 16 threads of row p
+        // are a half-warp: shuffles), dK = Diag(beta) dA into DTM.
         for (int c = tid; c < DK; c += kThreads) {
             float acc = DGC[c];
             for (int g = 0; g < CH / 4; ++g) acc += DGP[g * DK + c];
             DGC[c] = acc;                     // both go to the last row's g
         }
-        for (int idx = tid; idx < CH * CH; idx += kThreads) {
-            const int r = idx / CH, m = idx % CH;
-            float acc = 0.f;
-            for (int i = 0; i <= (r < m ? r : m); ++i) acc = fmaf(DTM[r * LC + i] * BT[i], TM[m * LC + i], acc);
-            XM[r * LC + m] = acc;
-        }
-        __syncthreads();
-        // dA = strict-lower(-T^T X); dbeta_r += sum_i dA_ri K_ri; dK = Diag(beta) dA (into DTM)
-        for (int idx = tid; idx < CH * CH; idx += kThreads) {
-            const int p = idx / CH, m = idx % CH;
+        if (tid < CH * CH) {
+            const int p = tid / CH, m = tid % CH;
             float acc = 0.f;
             if (m < p)
                 for (int r = p; r < CH; ++r) acc = fmaf(TM[r * LC + p], XM[r * LC + m], acc);
-            DTM[p * LC + m] = -acc;              // dA, strictly lower (zero elsewhere)
-        }
-        __syncthreads();
-        if (tid < CH) {
-            const int r = tid;
-            float acc = 0.f;
-            for (int i = 0; i < r; ++i) acc = fmaf(DTM[r * LC + i], KM[r * LC + i], acc);
-            DB[r] += acc;
-        }
-        __syncthreads();
-        for (int idx = tid; idx < CH * CH; idx += kThreads) {
-            const int r = idx / CH, i = idx % CH;
-            DTM[r * LC + i] *= BT[r];            // dK
+            const float da = -acc;               // dA, strictly lower (zero elsewhere)
+            float t = m < p ? da * KM[p * LC + m] : 0.f;
+#pragma unroll
+            for (int o = 8; o > 0; o >>= 1) t += __shfl_xor_sync(0xffffffffu, t, o);
+            if (m == 0) DB[p] += t;
+            DTM[p * LC + m] = da * BT[p];        // dK
         }
         __syncthreads();
         if (fast) {
