@@ -38,6 +38,11 @@ constexpr int kC = 16;
 // factors D[r][i][c] = gamma_r / gamma_i as products of gamma_r and 1 / gamma_i, both in
 // [1, e^80] or [e^-80, 1]: K, P and their gradients through D become plain small products.
 constexpr float kFastGammaMin = 1.8048513e-35f;   // e^-80
+// Floats of a checkpoint block: state [dk][dvh], r and u [kC][dvh], K and T [kC][kC + 1] (padded as
+// in shared memory).
+__host__ __device__ constexpr size_t kBlockFloats(int dk, int dvh) {
+    return (size_t)(dk + 2 * kC) * dvh + 2 * kC * (kC + 1);
+}
 static_assert(kThreads == 32 * kC, "the K / P and gradient passes map warp w to row or column w, lane to a channel group");
 static_assert(2 * 128 + 128 < kThreads - kC, "gradient products, rowsum, X and dbeta on separate threads");
 static_assert(kC * kC <= kThreads && kC == 16, "dA: one thread per entry, a row per half-warp");
@@ -58,7 +63,7 @@ struct BwdLayout {
     static constexpr int V = DS + DK * LV, R = V + kC * LV, U = R + kC * LV, DO = U + kC * LV,
                          DU = DO + kC * LV, DR = DU + kC * LV;
     // [kC][LC] arrays
-    static constexpr int KM = DR + kC * LV, TM = KM + kC * LC, PM = TM + kC * LC, DPM = PM + kC * LC,
+    static constexpr int KM = DR + kC * LV, TM = KM + kC * LC, PM = TM + kC * LC, DPM = PM + kC * LC,   // K, T adjacent
                          DTM = DPM + kC * LC, XM = DTM + kC * LC;
     static constexpr int GC = XM + kC * LC, BT = GC + DK, DB = BT + kC, DGC = DB + kC;
     static constexpr int DGP = DGC + DK;      // [kThreads / DK][DK] partial last-row g terms; while
@@ -79,8 +84,8 @@ struct BwdArgs {
     const float *dS_final;          // [N, H, dk, dv] or NULL
     void *dv_out;                   // [T_total, H, dv] dtype
     float *dS0;                     // [N, H, dk, dv] or NULL
-    float *ckpt;                    // checkpoints: [max_chunks][H][nsplit] blocks of (dk + 2 kC) x dvh:
-                                    // the chunk-start state, then the chunk's r and u
+    float *ckpt;                    // checkpoints: [max_chunks][H][nsplit] blocks of kBlockFloats(dk, dvh):
+                                    // the chunk-start state, the chunk's r and u, then K and T
     float *part;                    // shares: [nsplit][T_total][H] x (3 dk + 1): dq, dk, dla, dbeta
     int64_t max_chunks;             // ceil(T_total / 16) + N with cu_seqlens, N ceil(T / 16) without
     int nsplit;
@@ -120,7 +125,7 @@ __global__ void __launch_bounds__(kThreads, 1) kda_chunk_bwd_kernel(BwdArgs b) {
     static_assert(RPT >= 1 && (CPT % 4 == 0 || CPT < 4) && R7 >= 1 && DK % 32 == 0 && DVH % 4 == 0,
                   "backward tiling");
     constexpr int NTU = (DVH / 2) * (DK / 16);   // threads of the state updates (2 columns x 16 rows)
-    static_assert(NTU <= kThreads, "state update tiling");
+    static_assert(NTU + DK + kC <= kThreads, "state update tiling; the gradient write-out beside it");
     extern __shared__ float sm[];
     float *Q = sm + L::Q, *Kk = sm + L::Kk, *AL = sm + L::AL, *GA = sm + L::GA, *KA = sm + L::KA;
     float *KG = sm + L::KG, *SQ = sm + L::SQ, *KK = sm + L::KK, *DQ = sm + L::DQ, *DKc = sm + L::DKc;
@@ -165,7 +170,7 @@ __global__ void __launch_bounds__(kThreads, 1) kda_chunk_bwd_kernel(BwdArgs b) {
     if (nch64 > b.max_chunks - base) nch64 = b.max_chunks - base;
     const int nch = (int)nch64;
     auto ckpt_block = [&](int ci) {
-        return b.ckpt + (((size_t)(base + ci) * H + h) * b.nsplit + split) * (size_t)(DK + 2 * CH) * DVH;
+        return b.ckpt + (((size_t)(base + ci) * H + h) * b.nsplit + split) * kBlockFloats(DK, DVH);
     };
     // Copies rows of `rows` x DVH floats (packed, from global) into a padded shared array.
     auto copy_in = [&](float *dst, const float *src, int rows) {
@@ -219,6 +224,8 @@ __global__ void __launch_bounds__(kThreads, 1) kda_chunk_bwd_kernel(BwdArgs b) {
     // Takes chunk c0's rows from the staging area (zeros / alpha = 1 / beta = 0 past the sequence
     // end; with_q: also q and dO), starts the copies of the next chunk (pf_nr rows from pf_c0,
     // none when pf_nr = 0), and forms the decay products and the chunk matrices K, T, P.
+    // The forward pass (form_ru) forms K, T, r and u; the backward pass (with_q) forms P and finds
+    // K, T, r and u in place (stored by the forward pass with the checkpoint, prefetched).
     auto chunk_terms = [&](int64_t c0, int nr, bool with_q, int64_t pf_c0, int pf_nr, bool pf_q,
                            bool form_ru) -> bool {
         cp_async_wait_all();
@@ -278,18 +285,18 @@ __global__ void __launch_bounds__(kThreads, 1) kda_chunk_bwd_kernel(BwdArgs b) {
             // parts).  Thread: (row r, column i).
             if (tid < CH * CH) {
                 const int r = tid / CH, i = tid % CH;
-                float sk = 0.f, sp = 0.f;
+                const float *A = form_ru ? KG : SQ;    // K in the forward pass, P in the backward
+                float acc = 0.f;
                 if (i <= r) {
 #pragma unroll 4
                     for (int c = 0; c < DK; c += 4) {
                         const float4 kk = ld4(KK + i * LK + c), rg = ld4(RGC + c);
                         const float4 ki = make_float4(kk.x * rg.x, kk.y * rg.y, kk.z * rg.z, kk.w * rg.w);
-                        sk = dot4(ld4(KG + r * LK + c), ki, sk);
-                        sp = dot4(ld4(SQ + r * LK + c), ki, sp);
+                        acc = dot4(ld4(A + r * LK + c), ki, acc);
                     }
                 }
-                KM[r * LC + i] = r > i ? sk : 0.f;
-                PM[r * LC + i] = r >= i ? sp : 0.f;
+                if (form_ru) KM[r * LC + i] = r > i ? acc : 0.f;
+                else PM[r * LC + i] = r >= i ? acc : 0.f;
             }
         } else {
         // K and P: warp i, lane = channel group cg of 32, carries running products down the rows
@@ -326,8 +333,8 @@ __global__ void __launch_bounds__(kThreads, 1) kda_chunk_bwd_kernel(BwdArgs b) {
             if (cg == 0) {
 #pragma unroll
                 for (int r = 0; r < CH; ++r) {
-                    KM[r * LC + i] = r > i ? sk[r] : 0.f;
-                    PM[r * LC + i] = r >= i ? scale * sp[r] : 0.f;
+                    if (form_ru) KM[r * LC + i] = r > i ? sk[r] : 0.f;
+                    if (with_q) PM[r * LC + i] = r >= i ? scale * sp[r] : 0.f;
                 }
             }
         }
@@ -335,7 +342,7 @@ __global__ void __launch_bounds__(kThreads, 1) kda_chunk_bwd_kernel(BwdArgs b) {
         // T = (I + Diag(beta) K)^{-1}, unit lower triangular: column i by forward substitution,
         // the column in registers (its entries above row i are zero, so the sums over m < i add
         // exact zeros before the first term, as if they started at m = i)
-        if (tid < CH) {
+        if (form_ru && tid < CH) {
             const int i = tid;
             float t[CH];
 #pragma unroll
@@ -403,6 +410,8 @@ __global__ void __launch_bounds__(kThreads, 1) kda_chunk_bwd_kernel(BwdArgs b) {
                 const float *from = row < CH ? R + row * LV + j : U + (row - CH) * LV + j;
                 *reinterpret_cast<float4 *>(ru + 4 * q) = ld4(from);
             }
+            float *kt = ru + 2 * CH * DVH;         // K and T, contiguous in shared memory
+            for (int q = tid; q < 2 * CH * LC / 4; q += kThreads) *reinterpret_cast<float4 *>(kt + 4 * q) = ld4(KM + 4 * q);
         }
         // S <- Diag(gamma_last) S + (k kappa)^T u, in place.  Thread: columns j, j + 1 and 16 rows
         // (each broadcast (k kappa) value feeds both columns).
@@ -589,6 +598,11 @@ __global__ void __launch_bounds__(kThreads, 1) kda_chunk_bwd_kernel(BwdArgs b) {
             DTM[p * LC + m] = da * BT[p];        // dK
         }
         __syncthreads();
+        if (ci > 0) {                          // K and T are not read again for this chunk
+            const float *kt = ckpt_block(ci - 1) + (DK + 2 * CH) * DVH;
+            for (int q = tid; q < 2 * CH * LC / 4; q += kThreads) cp_async16(KM + 4 * q, kt + 4 * q);
+            cp_async_commit();
+        }
         if (fast) {
             // through D = gamma_r / gamma_i in K and P, as products: for row / column x and channel c
             //   adk = (1 / gamma_x) sum_r (dP_rx (s q gamma)_r + dK_rx (k gamma)_r),  adg = -k_x adk,
@@ -674,8 +688,10 @@ __global__ void __launch_bounds__(kThreads, 1) kda_chunk_bwd_kernel(BwdArgs b) {
             }
         }
         __syncthreads();
-        // dlog_alpha = reverse cumulative sum of dg; write this half's share of the rows
-        for (int c = tid; c < DK; c += kThreads) {
+        // dlog_alpha = reverse cumulative sum of dg; write this half's share of the rows (on the
+        // threads past those of the dS update below, which runs at the same time)
+        if (tid >= NTU && tid < NTU + DK) {
+            const int c = tid - NTU;
             float acc = DGC[c];                    // the last row's extra g terms
             for (int r = CH - 1; r >= 0; --r) {
                 acc += DG[r * LK + c];
@@ -688,7 +704,10 @@ __global__ void __launch_bounds__(kThreads, 1) kda_chunk_bwd_kernel(BwdArgs b) {
                 }
             }
         }
-        if (tid < nr) b.part[part_index(b, split, (size_t)(c0 + tid) * H + h, DK) + 3 * DK] = DB[tid];
+        if (tid >= NTU + DK && tid < NTU + DK + nr) {
+            const int r = tid - NTU - DK;
+            b.part[part_index(b, split, (size_t)(c0 + r) * H + h, DK) + 3 * DK] = DB[r];
+        }
         // dS for the previous chunk, in place: (s q gamma)^T dO + Diag(gamma_last) dS' - (k gamma)^T dr.
         // Thread: columns j, j + 1 and 16 rows.
         if (tid < NTU) {
@@ -810,7 +829,7 @@ int64_t bwd_max_chunks(const KdaChunkArgs &a) {
 
 size_t kda_chunk_bwd_workspace_bytes(const KdaChunkArgs &a) {
     const int nsplit = a.dv > 64 ? a.dv / 64 : 1, dvh = a.dv / nsplit;
-    const size_t ck = (size_t)bwd_max_chunks(a) * a.H * nsplit * (a.dk + 2 * kC) * dvh * sizeof(float);
+    const size_t ck = (size_t)bwd_max_chunks(a) * a.H * nsplit * kBlockFloats(a.dk, dvh) * sizeof(float);
     const size_t part = (size_t)nsplit * a.T_total * a.H * (3 * (size_t)a.dk + 1) * sizeof(float);
     return ((ck + 255) & ~(size_t)255) + part;
 }
@@ -827,7 +846,7 @@ cudaError_t kda_launch_chunk_bwd(const KdaChunkArgs &a, int dtype, const void *d
     b.nsplit = a.dv > 64 ? a.dv / 64 : 1;
     const int dvh = a.dv / b.nsplit;
     b.max_chunks = bwd_max_chunks(a);
-    const size_t ck = (size_t)b.max_chunks * a.H * b.nsplit * (a.dk + 2 * kC) * dvh * sizeof(float);
+    const size_t ck = (size_t)b.max_chunks * a.H * b.nsplit * kBlockFloats(a.dk, dvh) * sizeof(float);
     b.ckpt = static_cast<float *>(ws);
     b.part = reinterpret_cast<float *>(static_cast<char *>(ws) + ((ck + 255) & ~(size_t)255));
     return dtype == 0 ? run<float>(b, dq, dk, dgate, dbeta, stream) : run<__nv_bfloat16>(b, dq, dk, dgate, dbeta, stream);
