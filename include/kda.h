@@ -209,9 +209,10 @@ int kda_chunk_fwd_ex(const void *q, const void *k, const void *v, int gate_kind,
  *   dbeta    [T_total, H]      fp32       written
  *   dS0      [N, H, dk, dv]    fp32 or NULL (not written)
  * Workspace: taken with cudaMallocAsync on `stream` from the default pool and freed on it
- * (the pool's release threshold is raised on first use, as for kda_chunk_fwd): one fp32 state
- * checkpoint per 16-token chunk per (head, 64-column d_v half) -- dk * dv * 4 bytes per 16
- * tokens per head -- plus (3 dk + 1) * 4 bytes per token-head per d_v half.
+ * (the pool's release threshold is raised on first use, as for kda_chunk_fwd): per 16-token
+ * chunk and (head, 64-column d_v half) one block of the chunk-start fp32 state and the chunk's
+ * terms the backward pass reuses -- ((dk + 32) * dvh + 544) * 4 bytes, dvh = min(dv, 64) --
+ * plus (3 dk + 1) * 4 bytes per token-head per d_v half.
  * Errors: as kda_chunk_fwd_ex (KDA_ERR_GATE for the fused form or any flag), KDA_ERR_NULL for
  * dO, dq, dk, dv, dbeta (or dgate with a decay form) NULL while T_total > 0, KDA_ERR_ALIAS
  * for an output overlapping an input or another output.
