@@ -21,13 +21,16 @@
 //   dlog_alpha = reverse cumulative sum of dg over the chunk's rows,
 //   dS = (s q gamma)^T dO + Diag(gamma_last) dS' - (k gamma)^T dr   (the previous chunk's dS').
 //
-// Every decay factor is a running product of alphas (no e^{+g}), as in the forward.
+// Every decay factor is a product of alphas (no e^{+g}): running products along the rows, or, in
+// a chunk whose decay stays within e^-80, gamma_r times kappa_i / gamma_last (both bounded).
 //
 // Kernels: (1) one CTA per (sequence, head, d_v half of up to 64 columns) walks the chunks
-// forward storing each chunk-start state (the checkpoints), then backward computing dv, dS0
-// and this half's share of dq, dk, dlog_alpha, dbeta; (2) a reduction adds the halves' shares in
-// a fixed order (every d_v-side sum enters those gradients linearly) and writes them in their
-// output types.  C = 16 keeps every chunk operand in shared memory at head size 128.
+// forward storing each chunk-start state (the checkpoints) with the chunk's r, u, K and T, then
+// backward computing dv, dS0 and this half's share of dq, dk, dlog_alpha, dbeta, each chunk's
+// inputs, checkpoint and stored terms prefetched (cp.async) while the chunk after it is
+// computed; (2) a reduction adds the halves' shares in a fixed order (every d_v-side sum enters
+// those gradients linearly) and writes them in their output types.  C = 16 keeps every chunk
+// operand in shared memory at head size 128.
 #include "kda_common.cuh"
 
 namespace {
@@ -403,7 +406,7 @@ __global__ void __launch_bounds__(kThreads, 1) kda_chunk_bwd_kernel(BwdArgs b) {
         // next: chunk ci + 1, or after the last one the backward pass's first chunk (the last)
         const int nx = ci + 1 < nch ? ci + 1 : nch - 1;
         chunk_terms(c0, nr, false, t0 + (int64_t)nx * CH, chunk_rows(nx), ci + 1 >= nch, true);
-        {   // the chunk's r and u beside its checkpoint, for the backward pass
+        {   // the chunk's r, u, K and T beside its checkpoint, for the backward pass
             float *ru = dst + DK * DVH;
             for (int q = tid; q < 2 * CH * DVH / 4; q += kThreads) {
                 const int row = 4 * q / DVH, j = 4 * q % DVH;
@@ -444,9 +447,10 @@ __global__ void __launch_bounds__(kThreads, 1) kda_chunk_bwd_kernel(BwdArgs b) {
     }
 
     // ---------------------------------------------------------------- backward
-    // Each chunk's checkpoint, r and u arrive by cp.async: the last chunk's checkpoint now (its r
-    // and u are still in place from the forward pass), every earlier chunk's once the chunk after
-    // it no longer reads S, R and U (below, after the gradient products).
+    // Each chunk's checkpoint, r, u, K and T arrive by cp.async: the last chunk's checkpoint now
+    // (its r, u, K and T are still in place from the forward pass), every earlier chunk's once the
+    // chunk after it no longer reads them (below: S, R, U after the gradient products, K and T after
+    // dA).
     if (nch > 0) {
         copy_in(S, ckpt_block(nch - 1), DK);
         cp_async_commit();
@@ -457,7 +461,6 @@ __global__ void __launch_bounds__(kThreads, 1) kda_chunk_bwd_kernel(BwdArgs b) {
         const bool fast = chunk_terms(c0, nr, true, c0 - CH, ci > 0 ? CH : 0, true, false);
 
         // du = P^T dO + (k kappa) dS', then dr = Diag(beta) T^T du (this half's dv rows).
-        // Thread: column j, RPT rows.
         {
             if (tid < 4 * DVH) {                   // du: thread column j, 4 rows
                 const int j = tid % DVH, i0 = (tid / DVH) * 4;
