@@ -804,6 +804,23 @@ def decode_pairs(dev_in, S0, device, kda_decode_step):
     return gpu_pair
 
 
+def e2e_groups(N: int, cu=None, max_groups: int = 4):
+    """The end-to-end path's sequence groups: up to ``max_groups`` contiguous ranges of the N
+    sequences, as (first, end, token slice, rebased cu_seqlens or None).  Token tensors lead with
+    the sequence axis (fixed length: the slice is over sequences) or are packed (the slice is the
+    group's token range and its cu_seqlens start at 0)."""
+    P = min(N, max_groups)
+    out = []
+    for g in range(P):
+        b0, b1 = N * g // P, N * (g + 1) // P
+        if cu is None:
+            out.append((b0, b1, slice(b0, b1), None))
+        else:
+            out.append((b0, b1, slice(int(cu[b0]), int(cu[b1])),
+                        (np.asarray(cu[b0:b1 + 1], dtype=np.int64) - int(cu[b0])).astype(np.int32)))
+    return out
+
+
 def run_e2e(args, name, device, stream, rank, return_outputs=False):
     """The same metric through the public call with pinned host buffers: every step copies its
     inputs host -> device, makes the call and copies its results back, all inside the timed
@@ -836,16 +853,13 @@ def run_e2e(args, name, device, stream, rank, return_outputs=False):
     # Decode keeps the recurrent state resident in HBM across steps (it is the model's
     # memory, not a step input): a step moves the new token's q, k, v and gates in and
     # its o out.  Prefill moves every input in and o plus the final states out.
-    P = min(N, 4)
-    bounds = [(N * g // P, N * (g + 1) // P) for g in range(P)]
     groups = []
-    for b0, b1 in bounds:
-        # token tensors lead with the sequence axis, or (packed) with the group's token range
-        sl = slice(b0, b1) if cu is None else slice(int(cu[b0]), int(cu[b1]))
+    plan = e2e_groups(N, cu)
+    bounds = [(b0, b1) for b0, b1, _, _ in plan]
+    for b0, b1, sl, cu_g in plan:
         hin = {k: (None if host.get(k) is None else host[k][sl]) for k in ("q", "k", "v", "log_alpha", "beta")}
         hin["S0"] = None if host.get("S0") is None else host["S0"][b0:b1]
-        hin["cu_seqlens"] = None if cu is None else \
-            torch.from_numpy((cu[b0:b1 + 1] - cu[b0]).astype(np.int32)).pin_memory()
+        hin["cu_seqlens"] = None if cu_g is None else torch.from_numpy(cu_g).pin_memory()
         g = {"in": hin, "dev": {k: (None if t is None else torch.empty_like(t, device=device))
                                 for k, t in hin.items()},
              "out_h": out_host[sl], "out_d": torch.empty_like(out_host[sl], device=device)}
@@ -899,7 +913,7 @@ def run_e2e(args, name, device, stream, rank, return_outputs=False):
     world = int(os.environ.get("WORLD_SIZE", 1))
     res = {"value": units * world / (ms / 1e3), "unit": "tokens/s", "ms_per_step": ms,
            "steps": steps, "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
-           "path": f"pinned host -> kda_* public call -> pinned host, the sequences in {P} groups on "
+           "path": f"pinned host -> kda_* public call -> pinned host, the sequences in {len(groups)} groups on "
                    "three streams (copies in, calls, copies out overlapping)"
                    + (" (decode state resident in HBM)" if name == "decode" else "")}
     return (res, host, out_host, S_host) if return_outputs else res

@@ -6,6 +6,7 @@ import os
 import subprocess
 import sys
 
+import numpy as np
 import pytest
 
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
@@ -187,3 +188,27 @@ def test_oracle_view_applies_the_gate_front_end():
     np.testing.assert_array_equal(v.beta, gates.sigmoid(inp.beta))
     s = make_form_inputs(2, 20, 2, 32, 32, "f32", 11, "scalar")
     assert bench.oracle_view(s).log_alpha.shape == (40, 2, 32)
+
+
+@pytest.mark.parametrize("N", [1, 3, 4, 8, 9])
+def test_e2e_groups_partition_the_batch(N):
+    """The end-to-end path's groups cover every sequence once, in order, and (packed tokens)
+    every token once, each group's cu_seqlens rebased to start at 0 with its own lengths."""
+    sys.path.insert(0, ROOT)
+    import bench
+    rng = np.random.default_rng(N)
+    lens = rng.integers(0, 50, size=N)
+    cu = np.concatenate([[0], np.cumsum(lens)]).astype(np.int32)
+    for packed in (False, True):
+        groups = bench.e2e_groups(N, cu if packed else None)
+        assert 1 <= len(groups) <= 4
+        assert groups[0][0] == 0 and groups[-1][1] == N
+        for (a0, a1, _, _), (b0, b1, _, _) in zip(groups, groups[1:]):
+            assert a1 == b0 and a0 < a1
+        for b0, b1, sl, cg in groups:
+            if not packed:
+                assert (sl.start, sl.stop) == (b0, b1) and cg is None
+            else:
+                assert (sl.start, sl.stop) == (int(cu[b0]), int(cu[b1]))
+                assert cg.dtype == np.int32 and cg[0] == 0 and len(cg) == b1 - b0 + 1
+                np.testing.assert_array_equal(np.diff(cg), lens[b0:b1])
