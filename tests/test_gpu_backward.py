@@ -133,3 +133,24 @@ def test_backward_is_deterministic():
     a, b = run_bwd(inp, dO, dSf), run_bwd(inp, dO, dSf)
     for name in a:
         np.testing.assert_array_equal(a[name], b[name])
+
+
+def test_backward_malformed_cu_seqlens_stay_in_bounds():
+    """Offsets that are not non-decreasing ([0, T, 0, T]: two clamped sequences over the same
+    tokens) ask for more checkpoint blocks than the workspace holds; each sequence's blocks are
+    capped to what is left, so the call completes without a device error (its gradients are
+    unspecified: two sequences write the same tokens' shares)."""
+    from gated_delta_rule_119_b200 import kda_chunk_bwd, kda_device_status
+    T, H = 512, 2
+    inp = make_form_inputs(1, T, H, 128, 128, "bf16", 780, "channel", state=True)
+    t = to_torch(inp)
+    packed = {k_: t[k_].reshape(T, *t[k_].shape[2:]) for k_ in ("q", "k", "v", "log_alpha", "beta")}
+    dO, _ = grad_inputs(inp, 781, final=False)
+    dO_t = storage_to_torch(dO, inp.dtype, "cuda").view(packed["v"].shape)
+    cu = torch.tensor([0, T, 0, T], dtype=torch.int32, device="cuda")
+    S0 = torch.cat([t["S0"]] * 3)
+    g = kda_chunk_bwd(packed["q"], packed["k"], packed["v"], packed["log_alpha"], packed["beta"], dO_t,
+                      S0, cu)
+    torch.cuda.synchronize()
+    assert kda_device_status() == 0
+    assert g["dv"].shape == packed["v"].shape
